@@ -1,0 +1,204 @@
+"""CPU oracle for the KV-cache append + attention path (TEST INFRASTRUCTURE ONLY).
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import this package.  The product path (the C-ABI library and
+its Python binding) never imports, links or executes anything here, and this
+package imports nothing from the product package.
+
+The arithmetic lives in ``rtv_oracle.c`` (plain C, fp32 steps one rounding at
+a time, fp64 attention); this module loads it with ctypes, and holds the ring
+bookkeeping, which is integer-only and written as an explicit slot map.
+
+Sources (page title, section):
+  * aidose.in, "Runway explains how it serves a 57B video model in real time",
+    third paragraph: rotary embedding and FP8 quantisation happen once, as a
+    frame enters the cache; the cache is a ring buffer advanced without
+    copying; attention runs over it.
+  * pttl.gr, section "Από οκτώ H100 σε τέσσερις", second paragraph: the same
+    write-time transformations and circular buffer; 240 attention calls per
+    step.
+Everything those pages leave open (RoPE split and base, E4M3, per-token-head
+scales, window W, pinned slot, key set and mask) is a reading taken from the
+workload definition; each is listed in the design notes.
+
+Parity status: every function here is pinned by tests under ``tests/`` that
+do not reuse its code (closed forms, invariants, an independent library
+routine, brute force on tiny inputs).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "rtv_oracle.c")
+_LIB_PATH = os.path.join(_HERE, "liboracle.so")
+
+GCC_FLAGS = ["-O2", "-ffp-contract=off", "-fno-fast-math", "-fopenmp", "-shared", "-fPIC",
+             "-Wall", "-Wextra"]
+
+
+def build(force: bool = False) -> str:
+    """Compile ``rtv_oracle.c`` into ``liboracle.so`` next to it (gcc)."""
+    if (not force and os.path.exists(_LIB_PATH)
+            and os.path.getmtime(_LIB_PATH) >= os.path.getmtime(_SRC)):
+        return _LIB_PATH
+    tmp = _LIB_PATH + f".tmp{os.getpid()}"
+    subprocess.check_call(["gcc", *GCC_FLAGS, "-o", tmp, _SRC, "-lm"])
+    os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    global _lib
+    if _lib is None:
+        _lib = ctypes.CDLL(build())
+        _declare(_lib)
+    return _lib
+
+
+_P = ctypes.c_void_p
+
+
+def _declare(L):
+    L.oracle_e4m3_decode.restype = ctypes.c_double
+    L.oracle_e4m3_decode.argtypes = [ctypes.c_uint8]
+    L.oracle_e4m3_encode.restype = ctypes.c_uint8
+    L.oracle_e4m3_encode.argtypes = [ctypes.c_float]
+    L.oracle_e4m3_near_boundary.restype = ctypes.c_uint8
+    L.oracle_e4m3_near_boundary.argtypes = [ctypes.c_float]
+    L.oracle_e4m3_encode_array.argtypes = [_P, ctypes.c_long, _P]
+    L.oracle_e4m3_near_boundary_array.argtypes = [_P, ctypes.c_long, _P]
+    L.oracle_e4m3_decode_array.argtypes = [_P, ctypes.c_long, _P]
+    L.oracle_rope3d_array.argtypes = [_P, _P, ctypes.c_long, ctypes.c_int, ctypes.c_int,
+                                      ctypes.c_int, ctypes.c_int, _P, ctypes.c_double]
+    L.oracle_quantize_rows.argtypes = [_P, ctypes.c_long, ctypes.c_int, _P, _P, _P]
+    L.oracle_append_tensor.argtypes = [_P, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                       ctypes.c_int, ctypes.c_int, ctypes.c_long, ctypes.c_int,
+                                       ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_double,
+                                       _P, _P, _P]
+    L.oracle_attend.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, _P, _P,
+                                ctypes.c_int, _P, _P, _P, _P, ctypes.c_int, _P, _P, _P]
+    L.oracle_num_threads.restype = ctypes.c_int
+
+
+def _ptr(a: np.ndarray | None):
+    if a is None:
+        return None
+    assert a.flags["C_CONTIGUOUS"]
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def num_threads() -> int:
+    return lib().oracle_num_threads()
+
+
+# ----------------------------------------------------------------- E4M3 --
+
+def e4m3_encode(y) -> np.ndarray:
+    """RNE, saturating, sign-keeping fp32 -> E4M3 code (uint8), elementwise."""
+    y = np.ascontiguousarray(y, dtype=np.float32)
+    out = np.empty(y.shape, dtype=np.uint8)
+    lib().oracle_e4m3_encode_array(_ptr(y), y.size, _ptr(out))
+    return out
+
+
+def e4m3_near_boundary(y) -> np.ndarray:
+    y = np.ascontiguousarray(y, dtype=np.float32)
+    out = np.empty(y.shape, dtype=np.uint8)
+    lib().oracle_e4m3_near_boundary_array(_ptr(y), y.size, _ptr(out))
+    return out
+
+
+def e4m3_decode(codes) -> np.ndarray:
+    codes = np.ascontiguousarray(codes, dtype=np.uint8)
+    out = np.empty(codes.shape, dtype=np.float64)
+    lib().oracle_e4m3_decode_array(_ptr(codes), codes.size, _ptr(out))
+    return out
+
+
+# ----------------------------------------------------------------- RoPE --
+
+def rope3d(x, split, pos, base: float = 10000.0) -> np.ndarray:
+    """x: [n, D] fp32; pos: [n, 3] integer (t, h, w) -> rotated [n, D] fp32."""
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    n, D = x.shape
+    n_t, n_h, n_w = split
+    assert n_t + n_h + n_w == D
+    pos = np.ascontiguousarray(pos, dtype=np.int64).reshape(n, 3)
+    y = np.empty_like(x)
+    lib().oracle_rope3d_array(_ptr(x), _ptr(y), n, D, n_t, n_h, n_w, _ptr(pos), float(base))
+    return y
+
+
+def quantize_rows(x):
+    """x: [n, D] fp32 -> (codes [n, D] u8, scales [n] f32, near_boundary [n, D] u8)."""
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    n, D = x.shape
+    codes = np.empty((n, D), np.uint8)
+    scales = np.empty(n, np.float32)
+    near = np.empty((n, D), np.uint8)
+    lib().oracle_quantize_rows(_ptr(x), n, D, _ptr(codes), _ptr(scales), _ptr(near))
+    return codes, scales, near
+
+
+# --------------------------------------------------------------- append --
+
+def append_tensor(x_bf16_bits, T: int, grid_w: int, t0: int, apply_rope: bool, split,
+                  base: float = 10000.0):
+    """One of Q/K/V for one chunk.
+
+    x_bf16_bits: uint16 [rows, H, D] (bf16 bit patterns), rows = n_frames * T.
+    Returns head-major codes [H, rows, D] u8, scales [H, rows] f32 and the
+    rounding-boundary mask [H, rows, D] u8.
+    """
+    x = np.ascontiguousarray(x_bf16_bits, dtype=np.uint16)
+    rows, H, D = x.shape
+    assert D <= 512 and rows % T == 0
+    n_t, n_h, n_w = split
+    codes = np.empty((H, rows, D), np.uint8)
+    scales = np.empty((H, rows), np.float32)
+    near = np.empty((H, rows, D), np.uint8)
+    lib().oracle_append_tensor(_ptr(x), rows, H, D, T, grid_w, int(t0), int(bool(apply_rope)),
+                               n_t, n_h, n_w, float(base), _ptr(codes), _ptr(scales), _ptr(near))
+    return codes, scales, near
+
+
+# ------------------------------------------------------------ attention --
+
+def attend(qc, sq, kc, sk, vc, sv, rows=None, want_psum: bool = False):
+    """fp64 attention of the chunk's queries over the gathered key set.
+
+    qc [H, M, D] u8, sq [H, M] f32; kc/vc [H, NK, D] u8, sk/sv [H, NK] f32
+    (keys already in logical frame order).  rows: optional query-row sample.
+    Returns out [n_rows, H, D] f64 (and psum [n_rows, H] if asked).
+    """
+    qc = np.ascontiguousarray(qc, np.uint8)
+    kc = np.ascontiguousarray(kc, np.uint8)
+    vc = np.ascontiguousarray(vc, np.uint8)
+    sq = np.ascontiguousarray(sq, np.float32)
+    sk = np.ascontiguousarray(sk, np.float32)
+    sv = np.ascontiguousarray(sv, np.float32)
+    H, M, D = qc.shape
+    NK = kc.shape[1]
+    assert kc.shape == (H, NK, D) and vc.shape == (H, NK, D) and D <= 512
+    if rows is not None:
+        rows = np.ascontiguousarray(rows, np.int32)
+        assert rows.min() >= 0 and rows.max() < M
+        nr = rows.size
+    else:
+        nr = M
+    out = np.empty((nr, H, D), np.float64)
+    psum = np.empty((nr, H), np.float64) if want_psum else None
+    lib().oracle_attend(H, D, M, _ptr(qc), _ptr(sq), NK, _ptr(kc), _ptr(sk), _ptr(vc), _ptr(sv),
+                        nr, _ptr(rows), _ptr(out), _ptr(psum))
+    return (out, psum) if want_psum else out
+
+
+from .ring import OracleRing, OracleCache  # noqa: E402,F401
