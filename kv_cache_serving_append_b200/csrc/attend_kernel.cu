@@ -1,0 +1,423 @@
+// attend_kernel.cu -- attention of a staged chunk over the ring-buffer KV cache:
+// FP8 E4M3 QK^T and f16 PV on tcgen05 tensor cores with TMEM accumulators,
+// online softmax in registers.
+//
+// Source of the operation: aidose.in, "Runway explains how it serves a 57B
+// video model in real time", third paragraph (attention over the cache whose
+// frames were rotated and quantised once, at write time); pttl.gr, section
+// "Από οκτώ H100 σε τέσσερις" (240 attention calls per step).  The key set
+// (pinned frame, window, chunk) and the 1/sqrt(D) softmax are the library's
+// definition, stated in rtv.h.
+//
+// One CTA = 128 query rows of one head; 8 warps:
+//   warp 0    TMA producer: Q tile once; per KV tile the K and V code tiles
+//             (ring slot, head, token tile) and their per-token scales.
+//   warp 1    TMEM owner and MMA issuer: S_b = Q K^T (kind::f8f6f4, E4M3 x
+//             E4M3 -> f32, two S buffers), then O += P_{b'} V16 (kind::f16,
+//             P from TMEM, V from shared memory).
+//   warps 2-3 widen the V code tile to f16 (exact) in the MN-major layout the
+//             PV MMA reads.
+//   warps 4-7 softmax, one query row per thread: s*scale_k, running max,
+//             exp2, row sum, P = p * scale_v / Sv in f16 into TMEM; lazy O
+//             rescaling only when the running max grows by more than 2^8.
+// Logical-to-physical frame order is resolved in the TMA coordinates: the
+// kernel receives the key set as a list of ring slots and addresses
+// (slot * H + head) directly -- no gather, no copy.
+//
+// V's per-token scale varies along PV's contraction dimension, so it is
+// folded into P.  Sv is a power of two at or above every V scale in the key
+// set (from the per-frame V-scale maxima the append kernel records), which
+// keeps P = p * scale_v / Sv <= 2^8 inside f16 range; O is multiplied back by
+// Sv / l at the end.
+//
+// Every mbarrier wait is bounded; on time-out a thread sets the error word,
+// leaves its loop, and the CTA drains its own async work before returning.
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_fp8.h>
+
+#include "rtv_internal.h"
+#include "sm100.cuh"
+
+namespace rtv {
+namespace {
+
+using namespace sm100;
+
+constexpr int kBM = 128;        // query rows per CTA
+constexpr int kBN = 128;        // keys per KV tile
+constexpr int kStages = 3;      // K/V code tile stages
+constexpr int kThreads = 256;
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO = 256, kColP0 = 384, kColP1 = 448;
+constexpr float kLazyRescaleLog2 = 8.0f;   // rescale O only when the max grows by > 2^8
+
+template <int D>
+struct Smem {
+    static constexpr int kTileBytes = kBM * D;            // one FP8 code tile (Q, K or V)
+    static constexpr int kV16Bytes = kBN * D * 2;          // one f16 V tile
+    alignas(1024) uint8_t q[kTileBytes];
+    alignas(1024) uint8_t k[kStages][kTileBytes];
+    alignas(1024) uint8_t v8[kStages][kTileBytes];
+    alignas(1024) uint8_t v16[2][kV16Bytes];
+    alignas(128) float sk[kStages][kBN];
+    alignas(128) float sv[kStages][kBN];
+    uint64_t q_full;
+    uint64_t k_full[kStages];
+    uint64_t kv_empty[kStages];
+    uint64_t s_full[2], s_free[2], p_ready[2], v16_ready[2], pv_done[2];
+    uint64_t o_done;
+    uint32_t tmem_base;
+    int failed;
+};
+
+__device__ __forceinline__ float ex2(float x)
+{
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// Bounded wait whose outcome is the same for every lane of the warp, so that
+// warp-collective tcgen05.ld/st never run with a partial warp.
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, long long limit)
+{
+    return __all_sync(0xffffffffu, mbar_wait(bar, parity, limit));
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+attend_kernel(const __grid_constant__ AttendParams p, const __grid_constant__ CUtensorMap map_q,
+              const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_v,
+              const __grid_constant__ CUtensorMap map_sk, const __grid_constant__ CUtensorMap map_sv)
+{
+    extern __shared__ uint8_t smem_raw[];
+    Smem<D>& sm = *reinterpret_cast<Smem<D>*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int q0 = blockIdx.x * kBM;
+    const int h = blockIdx.y;
+    const int H = p.H;
+    const int n_tiles = p.n_frames_keys * p.tiles_per_frame;
+    const long long limit = p.wait_limit;
+
+    if (threadIdx.x == 0) {
+        mbar_init(&sm.q_full, 1);
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&sm.k_full[s], 1);
+            mbar_init(&sm.kv_empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&sm.s_full[b], 1);
+            mbar_init(&sm.s_free[b], 128);
+            mbar_init(&sm.p_ready[b], 128);
+            mbar_init(&sm.v16_ready[b], 64);
+            mbar_init(&sm.pv_done[b], 1);
+        }
+        mbar_init(&sm.o_done, 1);
+        sm.failed = 0;
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(&sm.tmem_base, kTmemCols);
+        tmem_relinquish();
+    }
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_desc(&map_q);
+        tma_prefetch_desc(&map_k);
+        tma_prefetch_desc(&map_v);
+        tma_prefetch_desc(&map_sk);
+        tma_prefetch_desc(&map_sv);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = sm.tmem_base;
+    bool fail = false;
+
+    if (warp == 0) {
+        // ------------------------------------------------------ producer --
+        if (lane == 0 && !p.debug_wait_fault) {
+            constexpr uint32_t kTileBytes = Smem<D>::kTileBytes;
+            mbar_arrive_expect_tx(&sm.q_full, kTileBytes);
+            tma_load_3d(sm.q, &map_q, &sm.q_full, 0, q0, h);
+            int issued = 0;
+            for (int j = 0; j < n_tiles; ++j) {
+                const int st = j % kStages;
+                if (j >= kStages &&
+                    !mbar_wait(&sm.kv_empty[st], ((j / kStages) - 1) & 1, limit)) {
+                    fail = true;
+                    break;
+                }
+                const int fi = j / p.tiles_per_frame;
+                const int t0 = (j - fi * p.tiles_per_frame) * kBN;
+                const int row = p.slot[fi] * H + h;
+                mbar_arrive_expect_tx(&sm.k_full[st], 2 * kTileBytes + 2 * kBN * 4);
+                tma_load_3d(sm.k[st], &map_k, &sm.k_full[st], 0, t0, row);
+                tma_load_3d(sm.v8[st], &map_v, &sm.k_full[st], 0, t0, row);
+                tma_load_2d(sm.sk[st], &map_sk, &sm.k_full[st], t0, row);
+                tma_load_2d(sm.sv[st], &map_sv, &sm.k_full[st], t0, row);
+                ++issued;
+            }
+            // drain: every copy this thread issued has landed before the CTA may exit
+            mbar_wait(&sm.q_full, 0, limit);
+            for (int j = issued - kStages; j < issued; ++j) {
+                if (j < 0) continue;
+                mbar_wait(&sm.k_full[j % kStages], (j / kStages) & 1, limit);
+            }
+        }
+    } else if (warp == 1) {
+        // ---------------------------------------------------- MMA issuer --
+        if (lane == 0) {
+            constexpr uint32_t kQK = idesc(kBM, kBN, 0, 0, 0, 0);        // E4M3 x E4M3 -> f32
+            constexpr uint32_t kPV = idesc(kBM, D, 0, 0, 0, 1);          // f16 x f16(MN) -> f32
+            constexpr uint32_t kSw = D == 128 ? kSwizzle128 : kSwizzle64;
+            constexpr uint32_t kSbo = D == 128 ? 1024 : 512;
+            const uint32_t q_addr = smem_u32(sm.q);
+            if (!mbar_wait(&sm.q_full, 0, limit)) fail = true;
+            for (int j = 0; j <= n_tiles && !fail; ++j) {
+                if (j < n_tiles) {
+                    const int st = j % kStages, b = j & 1;
+                    if (!mbar_wait(&sm.k_full[st], (j / kStages) & 1, limit)) { fail = true; break; }
+                    if (j >= 2 && !mbar_wait(&sm.s_free[b], ((j >> 1) - 1) & 1, limit)) { fail = true; break; }
+                    tc_fence_after();
+                    const uint32_t k_addr = smem_u32(sm.k[st]);
+                    const uint32_t d_s = tmem + (b ? kColS1 : kColS0);
+#pragma unroll
+                    for (int kk = 0; kk < D / 32; ++kk)
+                        mma_f8_ss(d_s, smem_desc(q_addr + kk * 32, 16, kSbo, kSw),
+                                  smem_desc(k_addr + kk * 32, 16, kSbo, kSw), kQK, kk > 0);
+                    tc_commit(&sm.s_full[b]);
+                }
+                if (j >= 1) {
+                    const int jp = j - 1, bp = jp & 1, stp = jp % kStages;
+                    if (!mbar_wait(&sm.p_ready[bp], (jp >> 1) & 1, limit)) { fail = true; break; }
+                    if (!mbar_wait(&sm.v16_ready[bp], (jp >> 1) & 1, limit)) { fail = true; break; }
+                    tc_fence_after();
+                    const uint32_t v_addr = smem_u32(sm.v16[bp]);
+                    const uint32_t a_p = tmem + (bp ? kColP1 : kColP0);
+#pragma unroll
+                    for (int kk = 0; kk < kBN / 16; ++kk)
+                        mma_f16_ts(tmem + kColO, a_p + kk * 8,
+                                   smem_desc(v_addr + kk * 2048, 16384, 1024, kSwizzle128), kPV,
+                                   (jp > 0 || kk > 0) ? 1u : 0u);
+                    tc_commit(&sm.pv_done[bp]);
+                    tc_commit(&sm.kv_empty[stp]);
+                }
+            }
+            tc_commit(&sm.o_done);
+            // drain: all MMAs issued by this thread complete before TMEM is freed
+            if (!mbar_wait(&sm.o_done, 0, limit)) fail = true;
+        }
+    } else if (warp < 4) {
+        // ------------------------------------------- V widening (FP8->f16) --
+        const int ct = threadIdx.x - 64;   // 0..63
+        constexpr int kChunks = D / 16;    // 16-byte chunks per key row
+        for (int j = 0; j < n_tiles; ++j) {
+            const int st = j % kStages, b = j & 1;
+            if (!warp_wait(&sm.k_full[st], (j / kStages) & 1, limit)) { fail = true; break; }
+            if (j >= 2 && !warp_wait(&sm.pv_done[b], ((j >> 1) - 1) & 1, limit)) { fail = true; break; }
+            const uint8_t* src = sm.v8[st];
+            uint8_t* dst = sm.v16[b];
+            for (int idx = ct; idx < kBN * kChunks; idx += 64) {
+                const int r = idx / kChunks, c = idx % kChunks;
+                const int sc = D == 128 ? (c ^ (r & 7)) : (c ^ ((r >> 1) & 3));
+                const uint4 raw = *reinterpret_cast<const uint4*>(src + r * D + sc * 16);
+                const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+                uint32_t o[8];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    __half2_raw lo = __nv_cvt_fp8x2_to_halfraw2(
+                        (__nv_fp8x2_storage_t)(w[i] & 0xffff), __NV_E4M3);
+                    __half2_raw hi = __nv_cvt_fp8x2_to_halfraw2(
+                        (__nv_fp8x2_storage_t)(w[i] >> 16), __NV_E4M3);
+                    o[2 * i] = (uint32_t)lo.x | ((uint32_t)lo.y << 16);
+                    o[2 * i + 1] = (uint32_t)hi.x | ((uint32_t)hi.y << 16);
+                }
+                // elements d = 16c .. 16c+15 -> n-block (16c)/64, 32-byte span (c%4) of the row
+                const int nb = (16 * c) / 64;
+                const int q0c = 2 * (c & 3);
+                uint8_t* rowp = dst + nb * (kBN * 128) + r * 128;
+                *reinterpret_cast<uint4*>(rowp + (((q0c) ^ (r & 7)) << 4)) =
+                    make_uint4(o[0], o[1], o[2], o[3]);
+                *reinterpret_cast<uint4*>(rowp + (((q0c + 1) ^ (r & 7)) << 4)) =
+                    make_uint4(o[4], o[5], o[6], o[7]);
+            }
+            fence_async_smem();   // generic-proxy writes -> visible to the MMA's async proxy
+            mbar_arrive(&sm.v16_ready[b]);
+        }
+    } else {
+        // --------------------------------------------------------- softmax --
+        const int row = threadIdx.x - 128;          // TMEM lane == query row in tile
+        const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+        const int qrow = q0 + row;
+        const bool row_ok = qrow < p.M;
+        const float sq = row_ok ? p.q_scales[(size_t)h * p.q_scale_pitch + qrow] : 0.f;
+        constexpr float kInvSqrtD = D == 128 ? 0.08838834764831845f : 0.125f;
+        const float c2 = sq * (1.4426950408889634f * kInvSqrtD);   // log2(e) / sqrt(D) * scale_q
+
+        // Sv: power of two >= every V scale of the key set
+        float vmax = 0.f;
+        for (int f = lane; f < p.n_frames_keys; f += 32)
+            vmax = fmaxf(vmax, __uint_as_float((uint32_t)(
+                                   p.v_scale_max[(size_t)p.slot[f] * H + h] & 0xffffffffull)));
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, o));
+        uint32_t ve = (__float_as_uint(vmax) >> 23) & 0xff;
+        if (__float_as_uint(vmax) & 0x7fffff) ve += 1;
+        if (vmax <= 0.f || ve < 2) ve = 127;
+        if (ve > 253) ve = 253;
+        const float Sv = __uint_as_float(ve << 23);
+        const float inv_Sv = __uint_as_float((254u - ve) << 23);
+
+        float m = -INFINITY;   // running max of s*scale_k (lazy)
+        float l = 0.f;
+        for (int j = 0; j < n_tiles && !fail; ++j) {
+            const int b = j & 1, st = j % kStages;
+            const int fi = j / p.tiles_per_frame;
+            const int nv = min(kBN, p.T - (j - fi * p.tiles_per_frame) * kBN);
+            if (!warp_wait(&sm.k_full[st], (j / kStages) & 1, limit)) { fail = true; break; }
+            if (!warp_wait(&sm.s_full[b], (j >> 1) & 1, limit)) { fail = true; break; }
+            tc_fence_after();
+            uint32_t sraw[kBN];
+            const uint32_t t_s = tmem + lane_off + (b ? kColS1 : kColS0);
+#pragma unroll
+            for (int c = 0; c < kBN / 32; ++c) tmem_ld32(t_s + c * 32, sraw + c * 32);
+            tc_wait_ld();
+            tc_fence_before();
+            mbar_arrive(&sm.s_free[b]);
+
+            const float* skp = sm.sk[st];
+            float u[kBN];
+            float mt = -INFINITY;
+#pragma unroll
+            for (int k = 0; k < kBN; ++k) {
+                u[k] = __uint_as_float(sraw[k]) * skp[k];
+                if (k < nv) mt = fmaxf(mt, u[k]);
+            }
+            const float m_new = fmaxf(m, mt);
+            if (m == -INFINITY) {
+                m = m_new;
+            } else if ((m_new - m) * c2 > kLazyRescaleLog2) {
+                const float alpha = ex2((m - m_new) * c2);
+                l *= alpha;
+                m = m_new;
+                // O holds PV up to tile j-1: wait for it, scale in place
+                if (!warp_wait(&sm.pv_done[(j - 1) & 1], ((j - 1) >> 1) & 1, limit)) { fail = true; break; }
+                tc_fence_after();
+                const uint32_t t_o = tmem + lane_off + kColO;
+#pragma unroll
+                for (int c = 0; c < D / 32; ++c) {
+                    uint32_t o[32];
+                    tmem_ld32(t_o + c * 32, o);
+                    tc_wait_ld();
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+                    tmem_st32(t_o + c * 32, o);
+                }
+                tc_wait_st();
+            }
+            const float mc = m * c2;
+            const float* svp = sm.sv[st];
+            uint32_t pk[kBN / 2];
+            float ls = 0.f;
+#pragma unroll
+            for (int k = 0; k < kBN; k += 2) {
+                float p0 = k < nv ? ex2(fmaf(u[k], c2, -mc)) : 0.f;
+                float p1 = k + 1 < nv ? ex2(fmaf(u[k + 1], c2, -mc)) : 0.f;
+                ls += p0 + p1;
+                __half2 hv = __floats2half2_rn(p0 * (svp[k] * inv_Sv), p1 * (svp[k + 1] * inv_Sv));
+                pk[k / 2] = *reinterpret_cast<uint32_t*>(&hv);
+            }
+            l += ls;
+            // P buffer b is free once PV(j-2) has completed
+            if (j >= 2 && !warp_wait(&sm.pv_done[b], ((j >> 1) - 1) & 1, limit)) { fail = true; break; }
+            tc_fence_after();
+            const uint32_t t_p = tmem + lane_off + (b ? kColP1 : kColP0);
+            tmem_st32(t_p, pk);
+            tmem_st32(t_p + 32, pk + 32);
+            tc_wait_st();
+            tc_fence_before();
+            mbar_arrive(&sm.p_ready[b]);
+        }
+        if (!fail && !warp_wait(&sm.o_done, 0, limit)) fail = true;
+        if (!fail) {
+            tc_fence_after();
+            const uint32_t t_o = tmem + lane_off + kColO;
+            const float norm = Sv / l;
+#pragma unroll
+            for (int c = 0; c < D / 32; ++c) {
+                uint32_t o[32];
+                tmem_ld32(t_o + c * 32, o);
+                tc_wait_ld();
+                if (row_ok) {
+                    if (p.out_bf16) {
+                        __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(p.out) +
+                                             ((size_t)qrow * H + h) * D + c * 32;
+#pragma unroll
+                        for (int i = 0; i < 32; i += 8) {
+                            uint4 w;
+                            __nv_bfloat162 a0 = __floats2bfloat162_rn(__uint_as_float(o[i]) * norm, __uint_as_float(o[i + 1]) * norm);
+                            __nv_bfloat162 a1 = __floats2bfloat162_rn(__uint_as_float(o[i + 2]) * norm, __uint_as_float(o[i + 3]) * norm);
+                            __nv_bfloat162 a2 = __floats2bfloat162_rn(__uint_as_float(o[i + 4]) * norm, __uint_as_float(o[i + 5]) * norm);
+                            __nv_bfloat162 a3 = __floats2bfloat162_rn(__uint_as_float(o[i + 6]) * norm, __uint_as_float(o[i + 7]) * norm);
+                            w.x = *reinterpret_cast<uint32_t*>(&a0);
+                            w.y = *reinterpret_cast<uint32_t*>(&a1);
+                            w.z = *reinterpret_cast<uint32_t*>(&a2);
+                            w.w = *reinterpret_cast<uint32_t*>(&a3);
+                            *reinterpret_cast<uint4*>(dst + i) = w;
+                        }
+                    } else {
+                        float* dst = reinterpret_cast<float*>(p.out) + ((size_t)qrow * H + h) * D + c * 32;
+#pragma unroll
+                        for (int i = 0; i < 32; i += 4)
+                            *reinterpret_cast<float4*>(dst + i) = make_float4(
+                                __uint_as_float(o[i]) * norm, __uint_as_float(o[i + 1]) * norm,
+                                __uint_as_float(o[i + 2]) * norm, __uint_as_float(o[i + 3]) * norm);
+                    }
+                }
+            }
+        }
+    }
+
+    if (fail) {
+        atomicOr(p.err, kErrTimeout);
+        sm.failed = 1;
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) {
+        __syncwarp();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+template <int D>
+cudaError_t launch(const AttendParams& p, const CUtensorMap* maps, cudaStream_t stream)
+{
+    const size_t smem = sizeof(Smem<D>) + 1024;
+    static bool configured = false;
+    if (!configured) {
+        cudaError_t e = cudaFuncSetAttribute(attend_kernel<D>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        configured = true;
+    }
+    dim3 grid((p.M + kBM - 1) / kBM, p.H);
+    attend_kernel<D><<<grid, kThreads, smem, stream>>>(p, maps[0], maps[1], maps[2], maps[3], maps[4]);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_attend(const AttendParams& p, const CUtensorMap* maps, int D, cudaStream_t stream)
+{
+    if (D == 128) return launch<128>(p, maps, stream);
+    if (D == 64) return launch<64>(p, maps, stream);
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace rtv

@@ -1,0 +1,215 @@
+"""Python binding of librtv (the C ABI in include/rtv.h).
+
+Argument marshalling only: every step of the append/attend path runs in the
+library's CUDA kernels.  PyTorch supplies device memory and streams.  There is
+no fallback: if ``librtv.so`` is missing or fails to load, importing this
+module raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "librtv.so")
+
+RTV_OK = 0
+RTV_ERR_INVALID_ARG = 1
+RTV_ERR_OOM = 2
+RTV_ERR_CUDA = 3
+RTV_ERR_STATE = 4
+RTV_ERR_TIMEOUT = 5
+RTV_ERR_UNSUPPORTED = 6
+RTV_OUT_F32 = 0
+RTV_OUT_BF16 = 1
+RTV_MAX_SLOTS = 64
+RTV_MAX_FRAMES_PER_CHUNK = 4
+
+
+class rtv_cache_config(ctypes.Structure):
+    _fields_ = [("n_layers", ctypes.c_int), ("n_heads", ctypes.c_int), ("head_dim", ctypes.c_int),
+                ("grid_h", ctypes.c_int), ("grid_w", ctypes.c_int),
+                ("max_frames_per_chunk", ctypes.c_int), ("window_frames", ctypes.c_int),
+                ("pinned_frames", ctypes.c_int), ("rope_t", ctypes.c_int),
+                ("rope_h", ctypes.c_int), ("rope_w", ctypes.c_int),
+                ("rope_base", ctypes.c_double)]
+
+
+class rtv_cache_state(ctypes.Structure):
+    _fields_ = [("frames_committed", ctypes.c_longlong),
+                ("generated_committed", ctypes.c_longlong),
+                ("pinned_committed", ctypes.c_int), ("head", ctypes.c_int),
+                ("n_slots", ctypes.c_int), ("n_visible", ctypes.c_int),
+                ("visible_slots", ctypes.c_int * RTV_MAX_SLOTS),
+                ("visible_frames", ctypes.c_longlong * RTV_MAX_SLOTS),
+                ("frame_of_slot", ctypes.c_longlong * RTV_MAX_SLOTS),
+                ("staged_layers", ctypes.c_int), ("staged_frames", ctypes.c_int)]
+
+
+class rtv_layer_layout(ctypes.Structure):
+    _fields_ = [("k_codes", ctypes.c_size_t), ("v_codes", ctypes.c_size_t),
+                ("k_scales", ctypes.c_size_t), ("v_scales", ctypes.c_size_t),
+                ("q_codes", ctypes.c_size_t), ("q_scales", ctypes.c_size_t),
+                ("v_scale_max", ctypes.c_size_t), ("scale_pitch", ctypes.c_int),
+                ("q_scale_pitch", ctypes.c_int)]
+
+
+_P = ctypes.c_void_p
+_S = ctypes.c_int
+_SIGS = {
+    "rtv_status_string": (ctypes.c_char_p, [_S]),
+    "rtv_cache_required_bytes": (_S, [ctypes.POINTER(rtv_cache_config), ctypes.POINTER(ctypes.c_size_t)]),
+    "rtv_cache_layer_layout": (_S, [ctypes.POINTER(rtv_cache_config), _S, ctypes.POINTER(rtv_layer_layout)]),
+    "rtv_cache_create": (_S, [ctypes.POINTER(rtv_cache_config), _P, ctypes.c_size_t, ctypes.POINTER(_P)]),
+    "rtv_cache_destroy": (_S, [_P]),
+    "rtv_cache_append": (_S, [_P, _S, _P, _P, _P, _S, _P]),
+    "rtv_attend": (_S, [_P, _S, _P, _S, _P]),
+    "rtv_cache_advance": (_S, [_P]),
+    "rtv_cache_get_state": (_S, [_P, ctypes.POINTER(rtv_cache_state)]),
+    "rtv_cache_device_buffer": (_S, [_P, ctypes.POINTER(_P), ctypes.POINTER(ctypes.c_size_t)]),
+    "rtv_cache_export": (_S, [_P, _S, _S, _P, _P, _P, _P, _P]),
+    "rtv_poll_error": (_S, [_P]),
+    "rtv_debug_set_wait_fault": (_S, [_P, _S, ctypes.c_longlong]),
+}
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"librtv.so not built ({LIB_PATH}); run "
+                          "`python -m kv_cache_serving_append_b200.build`")
+    L = ctypes.CDLL(LIB_PATH)
+    for name, (res, args) in _SIGS.items():
+        fn = getattr(L, name)
+        fn.restype = res
+        fn.argtypes = args
+    return L
+
+
+lib = _load()
+
+
+class RtvError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {status_string(status)} ({status})")
+
+
+def status_string(status: int) -> str:
+    return lib.rtv_status_string(status).decode()
+
+
+def check(status: int, what: str) -> None:
+    if status != RTV_OK:
+        raise RtvError(status, what)
+
+
+def make_config(cfg: dict) -> rtv_cache_config:
+    return rtv_cache_config(cfg["n_layers"], cfg["n_heads"], cfg["head_dim"], cfg["grid_h"],
+                            cfg["grid_w"], cfg["max_frames_per_chunk"], cfg["window_frames"],
+                            cfg["pinned_frames"], cfg["rope_t"], cfg["rope_h"], cfg["rope_w"],
+                            float(cfg.get("rope_base", 10000.0)))
+
+
+def required_bytes(cfg: dict) -> int:
+    c = make_config(cfg)
+    n = ctypes.c_size_t()
+    check(lib.rtv_cache_required_bytes(ctypes.byref(c), ctypes.byref(n)), "rtv_cache_required_bytes")
+    return n.value
+
+
+def layer_layout(cfg: dict, layer: int) -> rtv_layer_layout:
+    c = make_config(cfg)
+    out = rtv_layer_layout()
+    check(lib.rtv_cache_layer_layout(ctypes.byref(c), layer, ctypes.byref(out)),
+          "rtv_cache_layer_layout")
+    return out
+
+
+def _stream_ptr(stream):
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr())
+
+
+class Cache:
+    """A cache whose device buffer is a torch uint8 tensor owned by this object."""
+
+    def __init__(self, cfg: dict, device=None):
+        import torch
+        self.cfg = dict(cfg)
+        self.device = torch.device(device or "cuda")
+        self.nbytes = required_bytes(cfg)
+        self.buffer = torch.empty(self.nbytes, dtype=torch.uint8, device=self.device)
+        self._c = make_config(cfg)
+        h = ctypes.c_void_p()
+        with torch.cuda.device(self.device):
+            check(lib.rtv_cache_create(ctypes.byref(self._c), _ptr(self.buffer), self.nbytes,
+                                       ctypes.byref(h)), "rtv_cache_create")
+        self.handle = h
+        self.T = cfg["grid_h"] * cfg["grid_w"]
+
+    def close(self):
+        if self.handle:
+            check(lib.rtv_cache_destroy(self.handle), "rtv_cache_destroy")
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    # -- the hot path ----------------------------------------------------
+    def append(self, layer: int, q, k, v, n_frames: int, stream=None) -> int:
+        return lib.rtv_cache_append(self.handle, layer, _ptr(q), _ptr(k), _ptr(v), n_frames,
+                                    _stream_ptr(stream))
+
+    def attend(self, layer: int, out, stream=None) -> int:
+        import torch
+        dt = RTV_OUT_BF16 if out.dtype == torch.bfloat16 else RTV_OUT_F32
+        if out.dtype not in (torch.bfloat16, torch.float32):
+            return RTV_ERR_INVALID_ARG
+        return lib.rtv_attend(self.handle, layer, _ptr(out), dt, _stream_ptr(stream))
+
+    def advance(self) -> int:
+        return lib.rtv_cache_advance(self.handle)
+
+    # -- inspection ------------------------------------------------------
+    def state(self) -> rtv_cache_state:
+        st = rtv_cache_state()
+        check(lib.rtv_cache_get_state(self.handle, ctypes.byref(st)), "rtv_cache_get_state")
+        return st
+
+    def poll_error(self) -> int:
+        return lib.rtv_poll_error(self.handle)
+
+    def set_wait_fault(self, enable: bool, limit_cycles: int = 0) -> int:
+        return lib.rtv_debug_set_wait_fault(self.handle, int(enable), limit_cycles)
+
+    def views(self, layer: int) -> dict:
+        """torch views of one layer's tensors inside the device buffer."""
+        import torch
+        L = layer_layout(self.cfg, layer)
+        cfg = self.cfg
+        H, D, T = cfg["n_heads"], cfg["head_dim"], self.T
+        S = cfg["pinned_frames"] + cfg["window_frames"] + cfg["max_frames_per_chunk"]
+        qr = cfg["max_frames_per_chunk"] * T
+        b = self.buffer
+
+        def sl(off, n, dtype):
+            return b[off:off + n * torch.empty((), dtype=dtype).element_size()].view(dtype)
+
+        return dict(
+            k_codes=sl(L.k_codes, S * H * T * D, torch.uint8).view(S, H, T, D),
+            v_codes=sl(L.v_codes, S * H * T * D, torch.uint8).view(S, H, T, D),
+            k_scales=sl(L.k_scales, S * H * L.scale_pitch, torch.float32).view(S, H, L.scale_pitch)[..., :T],
+            v_scales=sl(L.v_scales, S * H * L.scale_pitch, torch.float32).view(S, H, L.scale_pitch)[..., :T],
+            q_codes=sl(L.q_codes, H * qr * D, torch.uint8).view(H, qr, D),
+            q_scales=sl(L.q_scales, H * L.q_scale_pitch, torch.float32).view(H, L.q_scale_pitch)[:, :qr],
+            v_scale_max=sl(L.v_scale_max, S * H, torch.int64).view(S, H),
+        )

@@ -1,0 +1,116 @@
+"""The C-ABI library loads on a CPU-only host, exports every symbol the header
+declares, and its host-only calls (sizes, layout, validation, status strings,
+the injected allocation failure) behave; no kernel is launched here."""
+import ctypes
+import os
+import re
+import subprocess
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "rtv.h")
+
+
+@pytest.fixture(scope="module")
+def rtv():
+    from kv_cache_serving_append_b200 import build
+    build.build()
+    from kv_cache_serving_append_b200 import rtv as mod
+    return mod
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"^(?:const char\*|rtv_status)\s+(rtv_\w+)\s*\(", text, re.M)))
+
+
+def test_header_declares_the_boundary():
+    syms = declared_symbols()
+    for name in ["rtv_cache_create", "rtv_cache_append", "rtv_attend", "rtv_cache_advance",
+                 "rtv_cache_destroy", "rtv_cache_get_state", "rtv_poll_error",
+                 "rtv_status_string", "rtv_cache_required_bytes", "rtv_cache_export"]:
+        assert name in syms
+
+
+def test_library_exports_every_declared_symbol(rtv):
+    lib = ctypes.CDLL(rtv.LIB_PATH)
+    missing = [s for s in declared_symbols() if not hasattr(lib, s)]
+    assert not missing
+    # and the binding wraps each of them under the same name
+    assert set(declared_symbols()) <= set(rtv._SIGS)
+    out = subprocess.run(["nm", "-D", "--defined-only", rtv.LIB_PATH], capture_output=True,
+                         text=True).stdout
+    exported = set(re.findall(r"\sT\s(rtv_\w+)", out))
+    assert set(declared_symbols()) <= exported
+
+
+def test_status_strings(rtv):
+    for s in range(7):
+        assert rtv.status_string(s)
+    assert rtv.status_string(5) == "kernel wait timed out"
+
+
+def test_required_bytes_and_layout(rtv):
+    from kv_cache_serving_append_b200 import configs
+    cfg = configs.get(3)
+    n = rtv.required_bytes(cfg)
+    H, D, T = 40, 128, 2992
+    S = 0 + 8 + 1
+    codes = 2 * S * H * T * D
+    assert n >= codes + H * T * D
+    assert n < codes * 1.2
+    L0 = rtv.layer_layout(cfg, 0)
+    for f in ("k_codes", "v_codes", "k_scales", "v_scales", "q_codes", "q_scales", "v_scale_max"):
+        assert getattr(L0, f) % 1024 == 0
+    assert L0.scale_pitch % 16 == 0 and L0.scale_pitch >= T
+    c4 = configs.get(4)
+    L1 = rtv.layer_layout(c4, 1)
+    L0 = rtv.layer_layout(c4, 0)
+    assert L1.k_codes - L0.k_codes == L1.q_codes - L0.q_codes > 0
+    assert rtv.required_bytes(c4) > 48 * 2 * S * H * T * D
+
+
+@pytest.mark.parametrize("change,status", [
+    (dict(head_dim=96, rope_t=32, rope_h=32, rope_w=32), 6),
+    (dict(rope_t=30, rope_h=50, rope_w=48), 6),
+    (dict(rope_t=31), 1),
+    (dict(rope_t=16), 1),
+    (dict(n_layers=0), 1),
+    (dict(pinned_frames=2), 1),
+    (dict(max_frames_per_chunk=5), 6),
+    (dict(window_frames=70), 6),
+    (dict(n_heads=300), 6),
+    (dict(rope_base=0.0), 1),
+])
+def test_invalid_configs_are_rejected(rtv, change, status):
+    from kv_cache_serving_append_b200 import configs
+    cfg = configs.get(2)
+    cfg.update(change)
+    c = rtv.make_config(cfg)
+    n = ctypes.c_size_t()
+    assert rtv.lib.rtv_cache_required_bytes(ctypes.byref(c), ctypes.byref(n)) == status
+
+
+def test_null_arguments(rtv):
+    assert rtv.lib.rtv_cache_required_bytes(None, None) == rtv.RTV_ERR_INVALID_ARG
+    assert rtv.lib.rtv_cache_destroy(None) == rtv.RTV_ERR_INVALID_ARG
+    assert rtv.lib.rtv_cache_advance(None) == rtv.RTV_ERR_INVALID_ARG
+    assert rtv.lib.rtv_attend(None, 0, None, 0, None) == rtv.RTV_ERR_INVALID_ARG
+    assert rtv.lib.rtv_cache_append(None, 0, None, None, None, 1, None) == rtv.RTV_ERR_INVALID_ARG
+    assert rtv.lib.rtv_poll_error(None) == rtv.RTV_ERR_INVALID_ARG
+
+
+def test_injected_allocation_failure_returns_oom():
+    """The out-of-memory path, injected on the host (no device call is made)."""
+    code = (
+        "import ctypes\n"
+        "from kv_cache_serving_append_b200 import rtv, configs\n"
+        "c = rtv.make_config(configs.get(1)); h = ctypes.c_void_p()\n"
+        "print(rtv.lib.rtv_cache_create(ctypes.byref(c), None, 0, ctypes.byref(h)), h.value)\n")
+    env = dict(os.environ, RTV_INJECT_ALLOC_FAILURE="1", PYTHONPATH=ROOT)
+    out = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True, env=env,
+                         cwd=ROOT, timeout=300)
+    assert out.returncode == 0, out.stderr
+    assert out.stdout.split() == ["2", "None"]
