@@ -298,9 +298,12 @@ attend_kernel(const __grid_constant__ AttendParams p, const __grid_constant__ CU
                 if (k < nv) mt = fmaxf(mt, u[k]);
             }
             const float m_new = fmaxf(m, mt);
-            if (m == -INFINITY) {
-                m = m_new;
-            } else if ((m_new - m) * c2 > kLazyRescaleLog2) {
+            if (j == 0) {
+                m = m_new;   // first tile: O not yet written
+            } else if (__any_sync(0xffffffffu, (m_new - m) * c2 > kLazyRescaleLog2)) {
+                // Warp-uniform decision: the wait and the TMEM load/store below
+                // are warp-collective.  Every lane moves to its own new max
+                // (alpha = 1 where it did not grow).
                 const float alpha = ex2((m - m_new) * c2);
                 l *= alpha;
                 m = m_new;
