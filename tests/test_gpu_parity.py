@@ -31,7 +31,7 @@ def run_full_compare(cfg_id, steps=None, check_attn_steps=None, rows_per_step=No
             if check_attn_steps is None or step in check_attn_steps:
                 rows = None
                 if rows_per_step:
-                    rows = sample_rows(F * R.T, rows_per_step, 1000 * step + layer)
+                    rows = sample_rows(F * R.T, rows_per_step, 1000 * (step + 1) + layer)
                 g, o = R.attend(layer, rows=rows, out_dtype=out_dtype)
                 mx, rl = attn_errors(g, o)
                 worst = (max(worst[0], mx), max(worst[1], rl))
