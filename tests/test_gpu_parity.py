@@ -94,8 +94,10 @@ def test_bf16_output_small(gpu):
             R.append(layer, step, 1)
         for layer in range(2):
             g, o = R.attend(layer, out_dtype=torch.bfloat16)
-            mx, rl = attn_errors(g, o)
-            # bf16 output adds at most half an ulp of bf16 (2^-9 relative)
-            assert mx <= ATOL_MAX and rl <= REL_L2
+            # the bf16 store adds up to half a bf16 ulp (2^-8 relative): the
+            # fp32 bound holds after that rounding
+            assert np.all(np.abs(g - o) <= ATOL_MAX + 2.0 ** -8 * np.abs(o))
+            _, rl = attn_errors(g, o)
+            assert rl <= REL_L2
         R.advance()
     R.cache.close()
