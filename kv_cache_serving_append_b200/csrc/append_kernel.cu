@@ -94,13 +94,30 @@ __device__ __forceinline__ void store_codes<4>(uint8_t* dst, const float* y, flo
     *reinterpret_cast<uint32_t*>(dst) = w0;
 }
 
+constexpr int kMaxRows = 32;   // token rows per block (host keeps rows_per_block <= this)
+
+template <int E>
+__device__ __forceinline__ void load_vec(const float* p, float* x)
+{
+#pragma unroll
+    for (int i = 0; i < E; i += 4) {
+        const float4 v = *reinterpret_cast<const float4*>(p + i);
+        x[i] = v.x; x[i + 1] = v.y; x[i + 2] = v.z; x[i + 3] = v.w;
+    }
+}
+
+__device__ __forceinline__ uint4 xor_vec(const uint4& v, uint32_t m) { return make_uint4(v.x ^ m, v.y ^ m, v.z ^ m, v.w ^ m); }
+__device__ __forceinline__ uint2 xor_vec(const uint2& v, uint32_t m) { return make_uint2(v.x ^ m, v.y ^ m); }
+
 // D = head_dim, E = D / 16 elements per lane.
 template <int D>
-__global__ void __launch_bounds__(kThreads) append_kernel(const __grid_constant__ AppendParams p)
+__global__ void __launch_bounds__(kThreads, 4) append_kernel(const __grid_constant__ AppendParams p)
 {
     constexpr int E = D / 16;
     using V = typename Vec<E>::T;
-    __shared__ float s_t[kMaxFrames][2][kMaxRopeHalf];
+    // Per local token row: the RoPE cos/sin this row needs, laid out along
+    // head_dim as [t cos | t sin | h cos | h sin | w cos | w sin] (half-widths).
+    __shared__ __align__(16) float s_tab[kMaxRows][D];
     __shared__ unsigned int s_vmax[kMaxHeads];
 
     const int tensor = blockIdx.y;             // 0 = Q, 1 = K, 2 = V
@@ -109,93 +126,91 @@ __global__ void __launch_bounds__(kThreads) append_kernel(const __grid_constant_
     const int n_rows = min(p.rows_per_block, p.T - tok0);
     const int H = p.H;
     const int n_items = n_rows * H;
+    const bool rope = tensor != 2;
+    const int ht = p.n_t / 2, hh = p.n_h / 2, hw = p.n_w / 2;
 
-    for (int i = threadIdx.x; i < kMaxFrames * 2 * kMaxRopeHalf; i += kThreads)
-        (&s_t[0][0][0])[i] = (&p.t_table[0][0][0])[i];
-    for (int i = threadIdx.x; i < H; i += kThreads)
-        s_vmax[i] = 0u;
+    for (int i = threadIdx.x; i < H; i += kThreads) s_vmax[i] = 0u;
+    if (rope) {
+        for (int i = threadIdx.x; i < n_rows * D; i += kThreads) {
+            const int r = i / D, d = i - r * D;
+            const int tok = tok0 + r;
+            float v;
+            if (d < 2 * ht) {
+                v = p.t_table[frame][d / ht][d % ht];
+            } else if (d < 2 * ht + 2 * hh) {
+                const int hp = tok / p.grid_w;
+                v = p.h_table[(size_t)hp * 2 * hh + (d - 2 * ht)];
+            } else {
+                const int wp = tok % p.grid_w;
+                v = p.w_table[(size_t)wp * 2 * hw + (d - 2 * ht - 2 * hh)];
+            }
+            s_tab[r][d] = v;
+        }
+    }
     __syncthreads();
 
     const int lane16 = threadIdx.x & 15;
     const int group = threadIdx.x >> 4;
     const int lane = threadIdx.x & 31;
-    const bool rope = tensor != 2;
 
-    // Fixed per lane: which RoPE segment its E elements fall in, the pair
-    // index of its first element, and which half of the pair it holds.
-    int seg = 0, seg_half = p.n_t / 2, seg_lo = 0;
+    // Fixed per lane: RoPE segment of its E elements, pair index of the
+    // first one, which half of the pair it holds, its partner lane, and where
+    // its cos/sin sit in the row table.
+    int seg_half = ht, seg_lo = 0, tab_lo = 0;
     if (lane16 * E >= p.n_t + p.n_h) {
-        seg = 2; seg_half = p.n_w / 2; seg_lo = p.n_t + p.n_h;
+        seg_half = hw; seg_lo = p.n_t + p.n_h; tab_lo = 2 * ht + 2 * hh;
     } else if (lane16 * E >= p.n_t) {
-        seg = 1; seg_half = p.n_h / 2; seg_lo = p.n_t;
+        seg_half = hh; seg_lo = p.n_t; tab_lo = 2 * ht;
     }
     const int in_seg = lane16 * E - seg_lo;
     const bool first_half = in_seg < seg_half;
     const int j0 = first_half ? in_seg : in_seg - seg_half;
     const int partner = (lane & 16) | (first_half ? lane16 + seg_half / E : lane16 - seg_half / E);
+    // x'[j] = x[j]c - x[j+n/2]s (first half) = x[j]c + (-x[j+n/2])s: the
+    // partner's value is negated by flipping its bf16 sign bits (exact).
+    const uint32_t neg_partner = first_half ? 0x80008000u : 0u;
+    const int c_off = tab_lo + j0, s_off = tab_lo + seg_half + j0;
 
     const uint16_t* src = p.src[tensor];
     const int row0 = frame * p.T + tok0;
 
-    // The loop bound is taken per warp (both half-warps iterate together) so
-    // that the full-warp shuffles below always have all 32 lanes present.
+    // Item it = (row it / H, head it % H), visited with stride kGroups; the
+    // (row, head) pair is advanced incrementally (no division per item).  The
+    // loop bound is taken per warp so the full-warp shuffles always have all
+    // 32 lanes present.
+    int r_it = group / H, h_it = group - (group / H) * H;
     for (int wbase = group & ~1; wbase < n_items; wbase += kGroups * kItems) {
         const int base = wbase + (group & 1);
         V raw[kItems];
+        int rr[kItems], hv[kItems];
 #pragma unroll
         for (int u = 0; u < kItems; ++u) {
-            const int it = base + u * kGroups;
+            rr[u] = r_it;
+            hv[u] = h_it;
             raw[u] = V{};
-            if (it < n_items) {
-                const int r = it / H, h = it - r * H;
-                const size_t off = ((size_t)(row0 + r) * H + h) * D + lane16 * E;
+            if (base + u * kGroups < n_items) {
+                const size_t off = ((size_t)(row0 + r_it) * H + h_it) * D + lane16 * E;
                 raw[u] = __ldcs(reinterpret_cast<const V*>(src + off));
             }
+            h_it += kGroups;
+            while (h_it >= H) { h_it -= H; ++r_it; }
         }
 #pragma unroll
         for (int u = 0; u < kItems; ++u) {
-            const int it = base + u * kGroups;
-            // uniform across the half-warp; shuffles below use the full warp,
-            // so both half-warps must take them together
-            const bool valid = it < n_items;
-            const int r = valid ? it / H : 0;
-            const int h = valid ? it - r * H : 0;
-            const int tok = tok0 + r;
-            float x[E], y[E];
-            unpack_bf16(raw[u], x);
+            const bool valid = base + u * kGroups < n_items;
+            const int r = valid ? rr[u] : 0;
+            const int h = hv[u];
+            float y[E];
+            unpack_bf16(raw[u], y);
             if (rope) {
-                V praw = shfl_vec(raw[u], partner);
-                float xp[E];
+                const V praw = xor_vec(shfl_vec(raw[u], partner), neg_partner);
+                float xp[E], cc[E], ss[E];
                 unpack_bf16(praw, xp);
-                const float* c;
-                const float* s;
-                if (seg == 0) {
-                    c = &s_t[frame][0][j0];
-                    s = &s_t[frame][1][j0];
-                } else if (seg == 1) {
-                    const int hp = tok / p.grid_w;
-                    c = p.h_table + (size_t)hp * 2 * seg_half + j0;
-                    s = c + seg_half;
-                } else {
-                    const int wp = tok % p.grid_w;
-                    c = p.w_table + (size_t)wp * 2 * seg_half + j0;
-                    s = c + seg_half;
-                }
-                float cc[E], ss[E];
+                load_vec<E>(&s_tab[r][c_off], cc);
+                load_vec<E>(&s_tab[r][s_off], ss);
 #pragma unroll
-                for (int e = 0; e < E; ++e) {
-                    cc[e] = c[e];   // generic loads: shared (frame axis) or global (L1-resident tables)
-                    ss[e] = s[e];
-                }
-#pragma unroll
-                for (int e = 0; e < E; ++e) {
-                    const float a = __fmul_rn(x[e], cc[e]);
-                    const float b = __fmul_rn(xp[e], ss[e]);
-                    y[e] = first_half ? __fsub_rn(a, b) : __fadd_rn(a, b);
-                }
-            } else {
-#pragma unroll
-                for (int e = 0; e < E; ++e) y[e] = x[e];
+                for (int e = 0; e < E; ++e)
+                    y[e] = __fadd_rn(__fmul_rn(y[e], cc[e]), __fmul_rn(xp[e], ss[e]));
             }
             float amax = 0.f;
 #pragma unroll
@@ -206,6 +221,7 @@ __global__ void __launch_bounds__(kThreads) append_kernel(const __grid_constant_
             if (!valid) continue;
             const float inv = amax > 0.f ? __fdiv_rn(448.f, amax) : 0.f;
             const float scale = __fdiv_rn(amax, 448.f);
+            const int tok = tok0 + r;
             uint8_t* dst;
             float* sdst;
             if (tensor == 0) {

@@ -78,6 +78,42 @@ __device__ __forceinline__ float ex2(float x)
     return y;
 }
 
+// Packed fp32 pairs (sm_100 f32x2 arithmetic: one instruction, two lanes of math).
+__device__ __forceinline__ uint64_t pack2(float a, float b)
+{
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+    return r;
+}
+__device__ __forceinline__ void unpack2(uint64_t r, float& a, float& b)
+{
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(r));
+}
+__device__ __forceinline__ uint64_t mul2(uint64_t a, uint64_t b)
+{
+    uint64_t r;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+__device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b)
+{
+    uint64_t r;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c)
+{
+    uint64_t r;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+    return r;
+}
+__device__ __forceinline__ float max3(float a, float b, float c)
+{
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+
 // Bounded wait whose outcome is the same for every lane of the warp, so that
 // warp-collective tcgen05.ld/st never run with a partial warp.
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, long long limit)
@@ -214,15 +250,24 @@ attend_kernel(const __grid_constant__ AttendParams p, const __grid_constant__ CU
     } else if (warp < 4) {
         // ------------------------------------------- V widening (FP8->f16) --
         const int ct = threadIdx.x - 64;   // 0..63
-        constexpr int kChunks = D / 16;    // 16-byte chunks per key row
         for (int j = 0; j < n_tiles; ++j) {
             const int st = j % kStages, b = j & 1;
             if (!warp_wait(&sm.k_full[st], (j / kStages) & 1, limit)) { fail = true; break; }
             if (j >= 2 && !warp_wait(&sm.pv_done[b], ((j >> 1) - 1) & 1, limit)) { fail = true; break; }
             const uint8_t* src = sm.v8[st];
             uint8_t* dst = sm.v16[b];
-            for (int idx = ct; idx < kBN * kChunks; idx += 64) {
-                const int r = idx / kChunks, c = idx % kChunks;
+            // A warp step covers 8 consecutive key rows x 4 chunk columns of one
+            // 64-element block: in every 8-lane shared-memory phase the 8 rows
+            // hit 8 different 16-byte bank groups, for the swizzled reads and
+            // for both swizzled writes.
+            constexpr int kNB = D / 64;                 // 64-element blocks per key row
+            const int wv = ct >> 5;                     // converter warp 0/1
+            const int rl = lane & 7, cq = lane >> 3;
+#pragma unroll 4
+            for (int combo = wv; combo < (kBN / 8) * kNB; combo += 2) {
+                const int r = (combo / kNB) * 8 + rl;
+                const int nb = combo % kNB;
+                const int c = nb * 4 + cq;                              // 16-byte chunk of the FP8 row
                 const int sc = D == 128 ? (c ^ (r & 7)) : (c ^ ((r >> 1) & 3));
                 const uint4 raw = *reinterpret_cast<const uint4*>(src + r * D + sc * 16);
                 const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
@@ -236,13 +281,11 @@ attend_kernel(const __grid_constant__ AttendParams p, const __grid_constant__ CU
                     o[2 * i] = (uint32_t)lo.x | ((uint32_t)lo.y << 16);
                     o[2 * i + 1] = (uint32_t)hi.x | ((uint32_t)hi.y << 16);
                 }
-                // elements d = 16c .. 16c+15 -> n-block (16c)/64, 32-byte span (c%4) of the row
-                const int nb = (16 * c) / 64;
-                const int q0c = 2 * (c & 3);
+                // elements d = 16c .. 16c+15 = block nb, bytes 32*cq .. 32*cq+31 of the row
                 uint8_t* rowp = dst + nb * (kBN * 128) + r * 128;
-                *reinterpret_cast<uint4*>(rowp + (((q0c) ^ (r & 7)) << 4)) =
+                *reinterpret_cast<uint4*>(rowp + (((2 * cq) ^ (r & 7)) << 4)) =
                     make_uint4(o[0], o[1], o[2], o[3]);
-                *reinterpret_cast<uint4*>(rowp + (((q0c + 1) ^ (r & 7)) << 4)) =
+                *reinterpret_cast<uint4*>(rowp + (((2 * cq + 1) ^ (r & 7)) << 4)) =
                     make_uint4(o[4], o[5], o[6], o[7]);
             }
             fence_async_smem();   // generic-proxy writes -> visible to the MMA's async proxy
@@ -258,22 +301,25 @@ attend_kernel(const __grid_constant__ AttendParams p, const __grid_constant__ CU
         constexpr float kInvSqrtD = D == 128 ? 0.08838834764831845f : 0.125f;
         const float c2 = sq * (1.4426950408889634f * kInvSqrtD);   // log2(e) / sqrt(D) * scale_q
 
-        // Sv: power of two >= every V scale of the key set
+        // Sv: power of two >= every V scale of the key set.  P = p * scale_v / Sv
+        // stays <= 2^8 in f16; dividing p by Sv is folded into the exponent
+        // (log2 Sv is an integer), so the row sum and O carry the same 1/Sv
+        // factor and O / l needs no correction.
         float vmax = 0.f;
         for (int f = lane; f < p.n_frames_keys; f += 32)
             vmax = fmaxf(vmax, __uint_as_float((uint32_t)(
                                    p.v_scale_max[(size_t)p.slot[f] * H + h] & 0xffffffffull)));
 #pragma unroll
         for (int o = 16; o >= 1; o >>= 1) vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, o));
-        uint32_t ve = (__float_as_uint(vmax) >> 23) & 0xff;
+        int ve = (int)((__float_as_uint(vmax) >> 23) & 0xff);
         if (__float_as_uint(vmax) & 0x7fffff) ve += 1;
-        if (vmax <= 0.f || ve < 2) ve = 127;
-        if (ve > 253) ve = 253;
-        const float Sv = __uint_as_float(ve << 23);
-        const float inv_Sv = __uint_as_float((254u - ve) << 23);
+        if (!(vmax > 0.f)) ve = 127;
+        ve = max(127 - 60, min(127 + 60, ve));
+        const float log2_sv = (float)(ve - 127);
 
-        float m = -INFINITY;   // running max of s*scale_k (lazy)
-        float l = 0.f;
+        float m = -INFINITY;   // running max of s * scale_k (lazy)
+        float l = 0.f;         // running sum of p / Sv
+        const uint64_t c2c2 = pack2(c2, c2);
         for (int j = 0; j < n_tiles && !fail; ++j) {
             const int b = j & 1, st = j % kStages;
             const int fi = j / p.tiles_per_frame;
@@ -281,22 +327,38 @@ attend_kernel(const __grid_constant__ AttendParams p, const __grid_constant__ CU
             if (!warp_wait(&sm.k_full[st], (j / kStages) & 1, limit)) { fail = true; break; }
             if (!warp_wait(&sm.s_full[b], (j >> 1) & 1, limit)) { fail = true; break; }
             tc_fence_after();
-            uint32_t sraw[kBN];
             const uint32_t t_s = tmem + lane_off + (b ? kColS1 : kColS0);
-#pragma unroll
-            for (int c = 0; c < kBN / 32; ++c) tmem_ld32(t_s + c * 32, sraw + c * 32);
-            tc_wait_ld();
-            tc_fence_before();
-            mbar_arrive(&sm.s_free[b]);
+            const float4* sk4 = reinterpret_cast<const float4*>(sm.sk[st]);
 
-            const float* skp = sm.sk[st];
-            float u[kBN];
-            float mt = -INFINITY;
+            // pass 1: row max of u = s * scale_k over the valid keys (S read
+            // from TMEM in 32-column chunks; nothing kept)
+            float mt0 = -INFINITY, mt1 = -INFINITY;
 #pragma unroll
-            for (int k = 0; k < kBN; ++k) {
-                u[k] = __uint_as_float(sraw[k]) * skp[k];
-                if (k < nv) mt = fmaxf(mt, u[k]);
+            for (int c = 0; c < kBN / 32; ++c) {
+                uint32_t sr[32];
+                tmem_ld32(t_s + c * 32, sr);
+                tc_wait_ld();
+#pragma unroll
+                for (int k4 = 0; k4 < 8; ++k4) {
+                    const float4 kk = sk4[c * 8 + k4];
+                    float a, bb, cc, d;
+                    unpack2(mul2(pack2(__uint_as_float(sr[4 * k4]), __uint_as_float(sr[4 * k4 + 1])),
+                                 pack2(kk.x, kk.y)), a, bb);
+                    unpack2(mul2(pack2(__uint_as_float(sr[4 * k4 + 2]), __uint_as_float(sr[4 * k4 + 3])),
+                                 pack2(kk.z, kk.w)), cc, d);
+                    const int k = c * 32 + 4 * k4;
+                    if (nv == kBN) {
+                        mt0 = max3(mt0, a, bb);
+                        mt1 = max3(mt1, cc, d);
+                    } else {
+                        if (k < nv) mt0 = fmaxf(mt0, a);
+                        if (k + 1 < nv) mt1 = fmaxf(mt1, bb);
+                        if (k + 2 < nv) mt0 = fmaxf(mt0, cc);
+                        if (k + 3 < nv) mt1 = fmaxf(mt1, d);
+                    }
+                }
             }
+            const float mt = fmaxf(mt0, mt1);
             const float m_new = fmaxf(m, mt);
             if (j == 0) {
                 m = m_new;   // first tile: O not yet written
@@ -311,7 +373,7 @@ attend_kernel(const __grid_constant__ AttendParams p, const __grid_constant__ CU
                 if (!warp_wait(&sm.pv_done[(j - 1) & 1], ((j - 1) >> 1) & 1, limit)) { fail = true; break; }
                 tc_fence_after();
                 const uint32_t t_o = tmem + lane_off + kColO;
-#pragma unroll
+#pragma unroll 1
                 for (int c = 0; c < D / 32; ++c) {
                     uint32_t o[32];
                     tmem_ld32(t_o + c * 32, o);
@@ -322,34 +384,64 @@ attend_kernel(const __grid_constant__ AttendParams p, const __grid_constant__ CU
                 }
                 tc_wait_st();
             }
-            const float mc = m * c2;
-            const float* svp = sm.sv[st];
-            uint32_t pk[kBN / 2];
-            float ls = 0.f;
-#pragma unroll
-            for (int k = 0; k < kBN; k += 2) {
-                float p0 = k < nv ? ex2(fmaf(u[k], c2, -mc)) : 0.f;
-                float p1 = k + 1 < nv ? ex2(fmaf(u[k + 1], c2, -mc)) : 0.f;
-                ls += p0 + p1;
-                __half2 hv = __floats2half2_rn(p0 * (svp[k] * inv_Sv), p1 * (svp[k + 1] * inv_Sv));
-                pk[k / 2] = *reinterpret_cast<uint32_t*>(&hv);
-            }
-            l += ls;
             // P buffer b is free once PV(j-2) has completed
             if (j >= 2 && !warp_wait(&sm.pv_done[b], ((j >> 1) - 1) & 1, limit)) { fail = true; break; }
             tc_fence_after();
+
+            // pass 2: p / Sv = 2^(u*c2 - m*c2 - log2 Sv); P = (p / Sv) * scale_v
+            // in f16 into TMEM, 64 keys (32 columns) at a time
+            const float neg = -(m * c2 + log2_sv);
+            const uint64_t neg2 = pack2(neg, neg);
+            const float4* sv4 = reinterpret_cast<const float4*>(sm.sv[st]);
             const uint32_t t_p = tmem + lane_off + (b ? kColP1 : kColP0);
-            tmem_st32(t_p, pk);
-            tmem_st32(t_p + 32, pk + 32);
+            uint64_t ls2 = pack2(0.f, 0.f);
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+                uint32_t sr[64];
+                tmem_ld32(t_s + half * 64, sr);
+                tmem_ld32(t_s + half * 64 + 32, sr + 32);
+                tc_wait_ld();
+                uint32_t pk[32];
+#pragma unroll
+                for (int k4 = 0; k4 < 16; ++k4) {
+                    const float4 kk = sk4[half * 16 + k4];
+                    const float4 vv = sv4[half * 16 + k4];
+#pragma unroll
+                    for (int hh = 0; hh < 2; ++hh) {
+                        const int kl = 4 * k4 + 2 * hh;         // key within this half
+                        const int k = half * 64 + kl;           // key within the tile
+                        const uint64_t u = mul2(pack2(__uint_as_float(sr[kl]), __uint_as_float(sr[kl + 1])),
+                                                hh ? pack2(kk.z, kk.w) : pack2(kk.x, kk.y));
+                        float x0, x1;
+                        unpack2(fma2(u, c2c2, neg2), x0, x1);
+                        float p0 = ex2(x0), p1 = ex2(x1);
+                        if (nv != kBN) {
+                            if (k >= nv) p0 = 0.f;
+                            if (k + 1 >= nv) p1 = 0.f;
+                        }
+                        const uint64_t pp = pack2(p0, p1);
+                        ls2 = add2(ls2, pp);
+                        float q0, q1;
+                        unpack2(mul2(pp, hh ? pack2(vv.z, vv.w) : pack2(vv.x, vv.y)), q0, q1);
+                        __half2 hv = __floats2half2_rn(q0, q1);
+                        pk[kl / 2] = *reinterpret_cast<uint32_t*>(&hv);
+                    }
+                }
+                tmem_st32(t_p + half * 32, pk);
+            }
+            float ls0, ls1;
+            unpack2(ls2, ls0, ls1);
+            l += ls0 + ls1;
             tc_wait_st();
             tc_fence_before();
+            mbar_arrive(&sm.s_free[b]);
             mbar_arrive(&sm.p_ready[b]);
         }
         if (!fail && !warp_wait(&sm.o_done, 0, limit)) fail = true;
         if (!fail) {
             tc_fence_after();
             const uint32_t t_o = tmem + lane_off + kColO;
-            const float norm = Sv / l;
+            const float norm = 1.f / l;
 #pragma unroll
             for (int c = 0; c < D / 32; ++c) {
                 uint32_t o[32];

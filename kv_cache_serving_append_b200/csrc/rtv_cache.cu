@@ -356,7 +356,7 @@ rtv_status rtv_cache_append(rtv_cache* c, int layer, const void* q, const void* 
     p.h_table = c->h_table;
     p.w_table = c->w_table;
     p.H = c->H; p.D = c->D; p.T = c->T; p.grid_w = c->cfg.grid_w; p.n_frames = n_frames;
-    p.rows_per_block = std::max(1, std::min(c->T, 256 / c->H));
+    p.rows_per_block = std::max(1, std::min(std::min(c->T, 32), 320 / c->H));
     p.blocks_per_frame = (c->T + p.rows_per_block - 1) / p.rows_per_block;
     p.q_rows = c->F_max * c->T;
     p.q_scale_pitch = L.q_scale_pitch;
