@@ -121,15 +121,101 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, long l
     return __all_sync(0xffffffffu, mbar_wait(bar, parity, limit));
 }
 
+// Pass 1 of a KV tile: row max of u = s * scale_k over the valid keys, S read
+// from TMEM in 32-column chunks.  kMask: tile with fewer than 128 valid keys.
+template <bool kMask>
+__device__ __forceinline__ float tile_row_max(uint32_t t_s, const float* sk, int nv)
+{
+    const float4* sk4 = reinterpret_cast<const float4*>(sk);
+    float mt0 = -INFINITY, mt1 = -INFINITY;
+#pragma unroll
+    for (int c = 0; c < kBN / 32; ++c) {
+        uint32_t sr[32];
+        tmem_ld32(t_s + c * 32, sr);
+        tc_wait_ld();
+#pragma unroll
+        for (int k4 = 0; k4 < 8; ++k4) {
+            const float4 kk = sk4[c * 8 + k4];
+            float a, b, cc, d;
+            unpack2(mul2(pack2(__uint_as_float(sr[4 * k4]), __uint_as_float(sr[4 * k4 + 1])),
+                         pack2(kk.x, kk.y)), a, b);
+            unpack2(mul2(pack2(__uint_as_float(sr[4 * k4 + 2]), __uint_as_float(sr[4 * k4 + 3])),
+                         pack2(kk.z, kk.w)), cc, d);
+            if (!kMask) {
+                mt0 = max3(mt0, a, b);
+                mt1 = max3(mt1, cc, d);
+            } else {
+                const int k = c * 32 + 4 * k4;
+                if (k < nv) mt0 = fmaxf(mt0, a);
+                if (k + 1 < nv) mt1 = fmaxf(mt1, b);
+                if (k + 2 < nv) mt0 = fmaxf(mt0, cc);
+                if (k + 3 < nv) mt1 = fmaxf(mt1, d);
+            }
+        }
+    }
+    return fmaxf(mt0, mt1);
+}
+
+// Pass 2 of a KV tile: p/Sv = 2^(u*c2 + neg), P = (p/Sv) * scale_v packed to
+// f16 pairs and stored into TMEM (64 keys = 32 columns at a time).  Returns
+// the tile's row sum of p/Sv.
+template <bool kMask>
+__device__ __forceinline__ float tile_make_p(uint32_t t_s, uint32_t t_p, const float* sk,
+                                             const float* sv, uint64_t c2c2, uint64_t neg2, int nv)
+{
+    const float4* sk4 = reinterpret_cast<const float4*>(sk);
+    const float4* sv4 = reinterpret_cast<const float4*>(sv);
+    uint64_t ls2 = pack2(0.f, 0.f);
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+        uint32_t sr[64];
+        tmem_ld32(t_s + half * 64, sr);
+        tmem_ld32(t_s + half * 64 + 32, sr + 32);
+        tc_wait_ld();
+        uint32_t pk[32];
+#pragma unroll
+        for (int k4 = 0; k4 < 16; ++k4) {
+            const float4 kk = sk4[half * 16 + k4];
+            const float4 vv = sv4[half * 16 + k4];
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+                const int kl = 4 * k4 + 2 * hh;
+                const uint64_t u = mul2(pack2(__uint_as_float(sr[kl]), __uint_as_float(sr[kl + 1])),
+                                        hh ? pack2(kk.z, kk.w) : pack2(kk.x, kk.y));
+                float x0, x1;
+                unpack2(fma2(u, c2c2, neg2), x0, x1);
+                float p0 = ex2(x0), p1 = ex2(x1);
+                if (kMask) {
+                    const int k = half * 64 + kl;
+                    if (k >= nv) p0 = 0.f;
+                    if (k + 1 >= nv) p1 = 0.f;
+                }
+                const uint64_t pp = pack2(p0, p1);
+                ls2 = add2(ls2, pp);
+                float q0, q1;
+                unpack2(mul2(pp, hh ? pack2(vv.z, vv.w) : pack2(vv.x, vv.y)), q0, q1);
+                __half2 hv = __floats2half2_rn(q0, q1);
+                pk[kl / 2] = *reinterpret_cast<uint32_t*>(&hv);
+            }
+        }
+        tmem_st32(t_p + half * 32, pk);
+    }
+    float a, b;
+    unpack2(ls2, a, b);
+    return a + b;
+}
+
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
 attend_kernel(const __grid_constant__ AttendParams p, const __grid_constant__ CUtensorMap map_q,
               const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_v,
               const __grid_constant__ CUtensorMap map_sk, const __grid_constant__ CUtensorMap map_sv)
 {
-    extern __shared__ uint8_t smem_raw[];
-    Smem<D>& sm = *reinterpret_cast<Smem<D>*>(
-        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    // 1024-byte alignment for the 128B-swizzled tiles, by offsetting the
+    // shared array itself (keeps the accesses in the shared address space)
+    const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
+    Smem<D>& sm = *reinterpret_cast<Smem<D>*>(smem_raw + pad);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -328,37 +414,9 @@ attend_kernel(const __grid_constant__ AttendParams p, const __grid_constant__ CU
             if (!warp_wait(&sm.s_full[b], (j >> 1) & 1, limit)) { fail = true; break; }
             tc_fence_after();
             const uint32_t t_s = tmem + lane_off + (b ? kColS1 : kColS0);
-            const float4* sk4 = reinterpret_cast<const float4*>(sm.sk[st]);
-
-            // pass 1: row max of u = s * scale_k over the valid keys (S read
-            // from TMEM in 32-column chunks; nothing kept)
-            float mt0 = -INFINITY, mt1 = -INFINITY;
-#pragma unroll
-            for (int c = 0; c < kBN / 32; ++c) {
-                uint32_t sr[32];
-                tmem_ld32(t_s + c * 32, sr);
-                tc_wait_ld();
-#pragma unroll
-                for (int k4 = 0; k4 < 8; ++k4) {
-                    const float4 kk = sk4[c * 8 + k4];
-                    float a, bb, cc, d;
-                    unpack2(mul2(pack2(__uint_as_float(sr[4 * k4]), __uint_as_float(sr[4 * k4 + 1])),
-                                 pack2(kk.x, kk.y)), a, bb);
-                    unpack2(mul2(pack2(__uint_as_float(sr[4 * k4 + 2]), __uint_as_float(sr[4 * k4 + 3])),
-                                 pack2(kk.z, kk.w)), cc, d);
-                    const int k = c * 32 + 4 * k4;
-                    if (nv == kBN) {
-                        mt0 = max3(mt0, a, bb);
-                        mt1 = max3(mt1, cc, d);
-                    } else {
-                        if (k < nv) mt0 = fmaxf(mt0, a);
-                        if (k + 1 < nv) mt1 = fmaxf(mt1, bb);
-                        if (k + 2 < nv) mt0 = fmaxf(mt0, cc);
-                        if (k + 3 < nv) mt1 = fmaxf(mt1, d);
-                    }
-                }
-            }
-            const float mt = fmaxf(mt0, mt1);
+            // pass 1: row max over the valid keys
+            const float mt = nv == kBN ? tile_row_max<false>(t_s, sm.sk[st], nv)
+                                       : tile_row_max<true>(t_s, sm.sk[st], nv);
             const float m_new = fmaxf(m, mt);
             if (j == 0) {
                 m = m_new;   // first tile: O not yet written
@@ -392,46 +450,9 @@ attend_kernel(const __grid_constant__ AttendParams p, const __grid_constant__ CU
             // in f16 into TMEM, 64 keys (32 columns) at a time
             const float neg = -(m * c2 + log2_sv);
             const uint64_t neg2 = pack2(neg, neg);
-            const float4* sv4 = reinterpret_cast<const float4*>(sm.sv[st]);
             const uint32_t t_p = tmem + lane_off + (b ? kColP1 : kColP0);
-            uint64_t ls2 = pack2(0.f, 0.f);
-#pragma unroll
-            for (int half = 0; half < 2; ++half) {
-                uint32_t sr[64];
-                tmem_ld32(t_s + half * 64, sr);
-                tmem_ld32(t_s + half * 64 + 32, sr + 32);
-                tc_wait_ld();
-                uint32_t pk[32];
-#pragma unroll
-                for (int k4 = 0; k4 < 16; ++k4) {
-                    const float4 kk = sk4[half * 16 + k4];
-                    const float4 vv = sv4[half * 16 + k4];
-#pragma unroll
-                    for (int hh = 0; hh < 2; ++hh) {
-                        const int kl = 4 * k4 + 2 * hh;         // key within this half
-                        const int k = half * 64 + kl;           // key within the tile
-                        const uint64_t u = mul2(pack2(__uint_as_float(sr[kl]), __uint_as_float(sr[kl + 1])),
-                                                hh ? pack2(kk.z, kk.w) : pack2(kk.x, kk.y));
-                        float x0, x1;
-                        unpack2(fma2(u, c2c2, neg2), x0, x1);
-                        float p0 = ex2(x0), p1 = ex2(x1);
-                        if (nv != kBN) {
-                            if (k >= nv) p0 = 0.f;
-                            if (k + 1 >= nv) p1 = 0.f;
-                        }
-                        const uint64_t pp = pack2(p0, p1);
-                        ls2 = add2(ls2, pp);
-                        float q0, q1;
-                        unpack2(mul2(pp, hh ? pack2(vv.z, vv.w) : pack2(vv.x, vv.y)), q0, q1);
-                        __half2 hv = __floats2half2_rn(q0, q1);
-                        pk[kl / 2] = *reinterpret_cast<uint32_t*>(&hv);
-                    }
-                }
-                tmem_st32(t_p + half * 32, pk);
-            }
-            float ls0, ls1;
-            unpack2(ls2, ls0, ls1);
-            l += ls0 + ls1;
+            l += nv == kBN ? tile_make_p<false>(t_s, t_p, sm.sk[st], sm.sv[st], c2c2, neg2, nv)
+                           : tile_make_p<true>(t_s, t_p, sm.sk[st], sm.sv[st], c2c2, neg2, nv);
             tc_wait_st();
             tc_fence_before();
             mbar_arrive(&sm.s_free[b]);
