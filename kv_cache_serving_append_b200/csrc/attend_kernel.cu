@@ -9,26 +9,35 @@
 // (pinned frame, window, chunk) and the 1/sqrt(D) softmax are the library's
 // definition, stated in rtv.h.
 //
-// One CTA = 128 query rows of one head; 8 warps:
-//   warp 0    TMA producer: Q tile once; per KV tile the K and V code tiles
-//             (ring slot, head, token tile) and their per-token scales.
-//   warp 1    TMEM owner and MMA issuer: S_b = Q K^T (kind::f8f6f4, E4M3 x
-//             E4M3 -> f32, two S buffers), then O += P_{b'} V16 (kind::f16,
-//             P from TMEM, V from shared memory).
-//   warps 2-3 widen the V code tile to f16 (exact) in the MN-major layout the
-//             PV MMA reads.
-//   warps 4-7 softmax, one query row per thread: s*scale_k, running max,
-//             exp2, row sum, P = p * scale_v / Sv in f16 into TMEM; lazy O
-//             rescaling only when the running max grows by more than 2^8.
+// One CTA = two 128-row query tiles of one head, sharing every K/V tile it
+// loads; 12 warps:
+//   warp 0     TMA producer: both Q tiles once; per KV tile the K and V code
+//              tiles at (ring slot * H + head, token tile) and their scales.
+//   warp 1     TMEM owner and MMA issuer.  Per query tile t and KV tile j:
+//              S_t = Q_t K_j^T (kind::f8f6f4, E4M3 x E4M3 -> f32 in TMEM),
+//              then O_t += P_t V16_j (kind::f16, P_t read from TMEM where it
+//              overwrote S_t, V16 from shared memory).  It issues whichever of
+//              the two tiles' next MMAs is ready, so one tile's softmax runs
+//              while the other tile's MMAs are on the tensor core.
+//   warps 2-3  widen the V code tile to f16 (exact) in the MN-major layout
+//              the PV MMA reads.
+//   warps 4-7  softmax of query tile 0, warps 8-11 of query tile 1; one query
+//              row per thread: s*scale_k, running max, exp2, row sum,
+//              P = p*scale_v/Sv in f16 written back over S; lazy O rescaling
+//              only when the running max grows by more than 2^8.
+// TMEM columns: S_0 [0,128), S_1 [128,256), O_0 [256,256+D), O_1 [384,384+D).
+// QK_t(j+1) is issued only once PV_t(j) has completed (its mbarrier), so the
+// P that PV_t(j) reads is never overwritten early and O_t is idle whenever
+// the softmax of tile t runs (the rescale needs no wait).
+//
 // Logical-to-physical frame order is resolved in the TMA coordinates: the
-// kernel receives the key set as a list of ring slots and addresses
-// (slot * H + head) directly -- no gather, no copy.
+// kernel receives the key set as a list of ring slots -- no gather, no copy.
 //
 // V's per-token scale varies along PV's contraction dimension, so it is
 // folded into P.  Sv is a power of two at or above every V scale in the key
-// set (from the per-frame V-scale maxima the append kernel records), which
-// keeps P = p * scale_v / Sv <= 2^8 inside f16 range; O is multiplied back by
-// Sv / l at the end.
+// set (from the per-frame V-scale maxima the append kernel records); P =
+// p*scale_v/Sv stays <= 2^8 inside f16 range, and 1/Sv is folded into the
+// exponent so the row sum carries the same factor and O/l needs none.
 //
 // Every mbarrier wait is bounded; on time-out a thread sets the error word,
 // leaves its loop, and the CTA drains its own async work before returning.
@@ -44,19 +53,22 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kBM = 128;        // query rows per CTA
+constexpr int kBM = 128;        // query rows per query tile
+constexpr int kQT = 2;          // query tiles per CTA
 constexpr int kBN = 128;        // keys per KV tile
 constexpr int kStages = 3;      // K/V code tile stages
-constexpr int kThreads = 256;
+constexpr int kThreads = 384;
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO = 256, kColP0 = 384, kColP1 = 448;
 constexpr float kLazyRescaleLog2 = 8.0f;   // rescale O only when the max grows by > 2^8
+
+__host__ __device__ constexpr uint32_t col_s(int t) { return 128u * t; }
+__host__ __device__ constexpr uint32_t col_o(int t) { return 256u + 128u * t; }
 
 template <int D>
 struct Smem {
     static constexpr int kTileBytes = kBM * D;            // one FP8 code tile (Q, K or V)
     static constexpr int kV16Bytes = kBN * D * 2;          // one f16 V tile
-    alignas(1024) uint8_t q[kTileBytes];
+    alignas(1024) uint8_t q[kQT][kTileBytes];
     alignas(1024) uint8_t k[kStages][kTileBytes];
     alignas(1024) uint8_t v8[kStages][kTileBytes];
     alignas(1024) uint8_t v16[2][kV16Bytes];
@@ -65,10 +77,10 @@ struct Smem {
     uint64_t q_full;
     uint64_t k_full[kStages];
     uint64_t kv_empty[kStages];
-    uint64_t s_full[2], s_free[2], p_ready[2], v16_ready[2], pv_done[2];
-    uint64_t o_done;
+    uint64_t s_full[kQT], p_ready[kQT], pv_done[kQT];
+    uint64_t v16_ready[2], tile_done[2];
+    uint64_t drain;
     uint32_t tmem_base;
-    int failed;
 };
 
 __device__ __forceinline__ float ex2(float x)
@@ -112,6 +124,14 @@ __device__ __forceinline__ float max3(float a, float b, float c)
     float r;
     asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
     return r;
+}
+// Four E4M3 codes (bytes of w) -> four f16 (exact), as two packed pairs.
+__device__ __forceinline__ void e4m3x4_to_f16x4(uint32_t w, uint32_t& lo, uint32_t& hi)
+{
+    asm("{\n\t.reg .b16 a, b;\n\tmov.b32 {a, b}, %2;\n\t"
+        "cvt.rn.f16x2.e4m3x2 %0, a;\n\tcvt.rn.f16x2.e4m3x2 %1, b;\n\t}"
+        : "=r"(lo), "=r"(hi)
+        : "r"(w));
 }
 
 // Bounded wait whose outcome is the same for every lane of the warp, so that
@@ -157,26 +177,26 @@ __device__ __forceinline__ float tile_row_max(uint32_t t_s, const float* sk, int
 }
 
 // Pass 2 of a KV tile: p/Sv = 2^(u*c2 + neg), P = (p/Sv) * scale_v packed to
-// f16 pairs and stored into TMEM (64 keys = 32 columns at a time).  Returns
-// the tile's row sum of p/Sv.
+// f16 pairs and written over S in TMEM: the 32 keys of S columns [32c, 32c+32)
+// become P columns [16c, 16c+16), which were all read before (in this chunk or
+// the previous one).  Returns the tile's row sum of p/Sv.
 template <bool kMask>
-__device__ __forceinline__ float tile_make_p(uint32_t t_s, uint32_t t_p, const float* sk,
-                                             const float* sv, uint64_t c2c2, uint64_t neg2, int nv)
+__device__ __forceinline__ float tile_make_p(uint32_t t_s, const float* sk, const float* sv,
+                                             uint64_t c2c2, uint64_t neg2, int nv)
 {
     const float4* sk4 = reinterpret_cast<const float4*>(sk);
     const float4* sv4 = reinterpret_cast<const float4*>(sv);
     uint64_t ls2 = pack2(0.f, 0.f);
 #pragma unroll
-    for (int half = 0; half < 2; ++half) {
-        uint32_t sr[64];
-        tmem_ld32(t_s + half * 64, sr);
-        tmem_ld32(t_s + half * 64 + 32, sr + 32);
+    for (int c = 0; c < kBN / 32; ++c) {
+        uint32_t sr[32];
+        tmem_ld32(t_s + c * 32, sr);
         tc_wait_ld();
-        uint32_t pk[32];
+        uint32_t pk[16];
 #pragma unroll
-        for (int k4 = 0; k4 < 16; ++k4) {
-            const float4 kk = sk4[half * 16 + k4];
-            const float4 vv = sv4[half * 16 + k4];
+        for (int k4 = 0; k4 < 8; ++k4) {
+            const float4 kk = sk4[c * 8 + k4];
+            const float4 vv = sv4[c * 8 + k4];
 #pragma unroll
             for (int hh = 0; hh < 2; ++hh) {
                 const int kl = 4 * k4 + 2 * hh;
@@ -186,7 +206,7 @@ __device__ __forceinline__ float tile_make_p(uint32_t t_s, uint32_t t_p, const f
                 unpack2(fma2(u, c2c2, neg2), x0, x1);
                 float p0 = ex2(x0), p1 = ex2(x1);
                 if (kMask) {
-                    const int k = half * 64 + kl;
+                    const int k = c * 32 + kl;
                     if (k >= nv) p0 = 0.f;
                     if (k + 1 >= nv) p1 = 0.f;
                 }
@@ -198,7 +218,7 @@ __device__ __forceinline__ float tile_make_p(uint32_t t_s, uint32_t t_p, const f
                 pk[kl / 2] = *reinterpret_cast<uint32_t*>(&hv);
             }
         }
-        tmem_st32(t_p + half * 32, pk);
+        tmem_st16(t_s + c * 16, pk);
     }
     float a, b;
     unpack2(ls2, a, b);
@@ -219,10 +239,11 @@ attend_kernel(const __grid_constant__ AttendParams p, const __grid_constant__ CU
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int q0 = blockIdx.x * kBM;
+    const int q0 = blockIdx.x * (kQT * kBM);
     const int h = blockIdx.y;
     const int H = p.H;
     const int n_tiles = p.n_frames_keys * p.tiles_per_frame;
+    const int n_qt = min(kQT, (p.M - q0 + kBM - 1) / kBM);   // query tiles with valid rows
     const long long limit = p.wait_limit;
 
     if (threadIdx.x == 0) {
@@ -231,15 +252,16 @@ attend_kernel(const __grid_constant__ AttendParams p, const __grid_constant__ CU
             mbar_init(&sm.k_full[s], 1);
             mbar_init(&sm.kv_empty[s], 1);
         }
-        for (int b = 0; b < 2; ++b) {
-            mbar_init(&sm.s_full[b], 1);
-            mbar_init(&sm.s_free[b], 128);
-            mbar_init(&sm.p_ready[b], 128);
-            mbar_init(&sm.v16_ready[b], 64);
-            mbar_init(&sm.pv_done[b], 1);
+        for (int t = 0; t < kQT; ++t) {
+            mbar_init(&sm.s_full[t], 1);
+            mbar_init(&sm.p_ready[t], 128);
+            mbar_init(&sm.pv_done[t], 1);
         }
-        mbar_init(&sm.o_done, 1);
-        sm.failed = 0;
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&sm.v16_ready[b], 64);
+            mbar_init(&sm.tile_done[b], 1);
+        }
+        mbar_init(&sm.drain, 1);
         fence_mbar_init();
     }
     if (warp == 1) {
@@ -263,8 +285,8 @@ attend_kernel(const __grid_constant__ AttendParams p, const __grid_constant__ CU
         // ------------------------------------------------------ producer --
         if (lane == 0 && !p.debug_wait_fault) {
             constexpr uint32_t kTileBytes = Smem<D>::kTileBytes;
-            mbar_arrive_expect_tx(&sm.q_full, kTileBytes);
-            tma_load_3d(sm.q, &map_q, &sm.q_full, 0, q0, h);
+            mbar_arrive_expect_tx(&sm.q_full, kQT * kTileBytes);
+            for (int t = 0; t < kQT; ++t) tma_load_3d(sm.q[t], &map_q, &sm.q_full, 0, q0 + t * kBM, h);
             int issued = 0;
             for (int j = 0; j < n_tiles; ++j) {
                 const int st = j % kStages;
@@ -297,58 +319,78 @@ attend_kernel(const __grid_constant__ AttendParams p, const __grid_constant__ CU
             constexpr uint32_t kPV = idesc(kBM, D, 0, 0, 0, 1);          // f16 x f16(MN) -> f32
             constexpr uint32_t kSw = D == 128 ? kSwizzle128 : kSwizzle64;
             constexpr uint32_t kSbo = D == 128 ? 1024 : 512;
-            const uint32_t q_addr = smem_u32(sm.q);
+            int qk_next[kQT] = {0, 0}, pv_next[kQT] = {0, 0};
             if (!mbar_wait(&sm.q_full, 0, limit)) fail = true;
-            for (int j = 0; j <= n_tiles && !fail; ++j) {
-                if (j < n_tiles) {
-                    const int st = j % kStages, b = j & 1;
-                    if (!mbar_wait(&sm.k_full[st], (j / kStages) & 1, limit)) { fail = true; break; }
-                    if (j >= 2 && !mbar_wait(&sm.s_free[b], ((j >> 1) - 1) & 1, limit)) { fail = true; break; }
-                    tc_fence_after();
-                    const uint32_t k_addr = smem_u32(sm.k[st]);
-                    const uint32_t d_s = tmem + (b ? kColS1 : kColS0);
+            long long last = clock64();
+            while (!fail) {
+                bool done = true, progressed = false;
+                for (int t = 0; t < n_qt; ++t) {
+                    if (pv_next[t] < n_tiles) done = false;
+                    // S_t = Q_t K_j^T once K_j has landed and PV_t(j-1) has completed
+                    int j = qk_next[t];
+                    if (j < n_tiles && j == pv_next[t] &&
+                        mbar_test(&sm.k_full[j % kStages], (j / kStages) & 1) &&
+                        (j == 0 || mbar_test(&sm.pv_done[t], (j - 1) & 1))) {
+                        tc_fence_after();
+                        const uint32_t q_addr = smem_u32(sm.q[t]);
+                        const uint32_t k_addr = smem_u32(sm.k[j % kStages]);
 #pragma unroll
-                    for (int kk = 0; kk < D / 32; ++kk)
-                        mma_f8_ss(d_s, smem_desc(q_addr + kk * 32, 16, kSbo, kSw),
-                                  smem_desc(k_addr + kk * 32, 16, kSbo, kSw), kQK, kk > 0);
-                    tc_commit(&sm.s_full[b]);
+                        for (int kk = 0; kk < D / 32; ++kk)
+                            mma_f8_ss(tmem + col_s(t), smem_desc(q_addr + kk * 32, 16, kSbo, kSw),
+                                      smem_desc(k_addr + kk * 32, 16, kSbo, kSw), kQK, kk > 0);
+                        tc_commit(&sm.s_full[t]);
+                        qk_next[t] = j + 1;
+                        progressed = true;
+                    }
+                    // O_t += P_t V_j once the softmax wrote P_t and V_j is widened
+                    j = pv_next[t];
+                    if (j < qk_next[t] && mbar_test(&sm.p_ready[t], j & 1) &&
+                        mbar_test(&sm.v16_ready[j & 1], (j >> 1) & 1)) {
+                        tc_fence_after();
+                        const uint32_t v_addr = smem_u32(sm.v16[j & 1]);
+#pragma unroll
+                        for (int kk = 0; kk < kBN / 16; ++kk)
+                            mma_f16_ts(tmem + col_o(t), tmem + col_s(t) + kk * 8,
+                                       smem_desc(v_addr + kk * 2048, 16384, 1024, kSwizzle128), kPV,
+                                       (j > 0 || kk > 0) ? 1u : 0u);
+                        tc_commit(&sm.pv_done[t]);
+                        pv_next[t] = j + 1;
+                        progressed = true;
+                        bool all = true;
+                        for (int u = 0; u < n_qt; ++u) all &= pv_next[u] > j;
+                        if (all) {   // every query tile consumed KV tile j
+                            tc_commit(&sm.kv_empty[j % kStages]);
+                            tc_commit(&sm.tile_done[j & 1]);
+                        }
+                    }
                 }
-                if (j >= 1) {
-                    const int jp = j - 1, bp = jp & 1, stp = jp % kStages;
-                    if (!mbar_wait(&sm.p_ready[bp], (jp >> 1) & 1, limit)) { fail = true; break; }
-                    if (!mbar_wait(&sm.v16_ready[bp], (jp >> 1) & 1, limit)) { fail = true; break; }
-                    tc_fence_after();
-                    const uint32_t v_addr = smem_u32(sm.v16[bp]);
-                    const uint32_t a_p = tmem + (bp ? kColP1 : kColP0);
-#pragma unroll
-                    for (int kk = 0; kk < kBN / 16; ++kk)
-                        mma_f16_ts(tmem + kColO, a_p + kk * 8,
-                                   smem_desc(v_addr + kk * 2048, 16384, 1024, kSwizzle128), kPV,
-                                   (jp > 0 || kk > 0) ? 1u : 0u);
-                    tc_commit(&sm.pv_done[bp]);
-                    tc_commit(&sm.kv_empty[stp]);
+                if (done) break;
+                if (progressed) {
+                    last = clock64();
+                } else {
+                    if (clock64() - last > limit) fail = true;
+                    __nanosleep(20);
                 }
             }
-            tc_commit(&sm.o_done);
             // drain: all MMAs issued by this thread complete before TMEM is freed
-            if (!mbar_wait(&sm.o_done, 0, limit)) fail = true;
+            tc_commit(&sm.drain);
+            if (!mbar_wait(&sm.drain, 0, limit)) fail = true;
         }
     } else if (warp < 4) {
         // ------------------------------------------- V widening (FP8->f16) --
-        const int ct = threadIdx.x - 64;   // 0..63
+        // A warp step covers 8 consecutive key rows x 4 chunk columns of one
+        // 64-element block: in every 8-lane shared-memory phase the 8 rows hit
+        // 8 different 16-byte bank groups, for the swizzled reads and for both
+        // swizzled writes.
+        constexpr int kNB = D / 64;                 // 64-element blocks per key row
+        const int wv = warp - 2;                    // converter warp 0/1
+        const int rl = lane & 7, cq = lane >> 3;
         for (int j = 0; j < n_tiles; ++j) {
             const int st = j % kStages, b = j & 1;
             if (!warp_wait(&sm.k_full[st], (j / kStages) & 1, limit)) { fail = true; break; }
-            if (j >= 2 && !warp_wait(&sm.pv_done[b], ((j >> 1) - 1) & 1, limit)) { fail = true; break; }
+            if (j >= 2 && !warp_wait(&sm.tile_done[b], ((j >> 1) - 1) & 1, limit)) { fail = true; break; }
             const uint8_t* src = sm.v8[st];
             uint8_t* dst = sm.v16[b];
-            // A warp step covers 8 consecutive key rows x 4 chunk columns of one
-            // 64-element block: in every 8-lane shared-memory phase the 8 rows
-            // hit 8 different 16-byte bank groups, for the swizzled reads and
-            // for both swizzled writes.
-            constexpr int kNB = D / 64;                 // 64-element blocks per key row
-            const int wv = ct >> 5;                     // converter warp 0/1
-            const int rl = lane & 7, cq = lane >> 3;
 #pragma unroll 4
             for (int combo = wv; combo < (kBN / 8) * kNB; combo += 2) {
                 const int r = (combo / kNB) * 8 + rl;
@@ -356,17 +398,11 @@ attend_kernel(const __grid_constant__ AttendParams p, const __grid_constant__ CU
                 const int c = nb * 4 + cq;                              // 16-byte chunk of the FP8 row
                 const int sc = D == 128 ? (c ^ (r & 7)) : (c ^ ((r >> 1) & 3));
                 const uint4 raw = *reinterpret_cast<const uint4*>(src + r * D + sc * 16);
-                const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
                 uint32_t o[8];
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    __half2_raw lo = __nv_cvt_fp8x2_to_halfraw2(
-                        (__nv_fp8x2_storage_t)(w[i] & 0xffff), __NV_E4M3);
-                    __half2_raw hi = __nv_cvt_fp8x2_to_halfraw2(
-                        (__nv_fp8x2_storage_t)(w[i] >> 16), __NV_E4M3);
-                    o[2 * i] = (uint32_t)lo.x | ((uint32_t)lo.y << 16);
-                    o[2 * i + 1] = (uint32_t)hi.x | ((uint32_t)hi.y << 16);
-                }
+                e4m3x4_to_f16x4(raw.x, o[0], o[1]);
+                e4m3x4_to_f16x4(raw.y, o[2], o[3]);
+                e4m3x4_to_f16x4(raw.z, o[4], o[5]);
+                e4m3x4_to_f16x4(raw.w, o[6], o[7]);
                 // elements d = 16c .. 16c+15 = block nb, bytes 32*cq .. 32*cq+31 of the row
                 uint8_t* rowp = dst + nb * (kBN * 128) + r * 128;
                 *reinterpret_cast<uint4*>(rowp + (((2 * cq) ^ (r & 7)) << 4)) =
@@ -379,129 +415,114 @@ attend_kernel(const __grid_constant__ AttendParams p, const __grid_constant__ CU
         }
     } else {
         // --------------------------------------------------------- softmax --
-        const int row = threadIdx.x - 128;          // TMEM lane == query row in tile
-        const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
-        const int qrow = q0 + row;
-        const bool row_ok = qrow < p.M;
-        const float sq = row_ok ? p.q_scales[(size_t)h * p.q_scale_pitch + qrow] : 0.f;
-        constexpr float kInvSqrtD = D == 128 ? 0.08838834764831845f : 0.125f;
-        const float c2 = sq * (1.4426950408889634f * kInvSqrtD);   // log2(e) / sqrt(D) * scale_q
+        const int t = (warp - 4) >> 2;              // query tile of this warpgroup
+        if (t < n_qt) {
+            const int row = (warp & 3) * 32 + lane;     // TMEM lane == query row in tile
+            const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+            const uint32_t t_s = tmem + lane_off + col_s(t);
+            const uint32_t t_o = tmem + lane_off + col_o(t);
+            const int qrow = q0 + t * kBM + row;
+            const bool row_ok = qrow < p.M;
+            const float sq = row_ok ? p.q_scales[(size_t)h * p.q_scale_pitch + qrow] : 0.f;
+            constexpr float kInvSqrtD = D == 128 ? 0.08838834764831845f : 0.125f;
+            const float c2 = sq * (1.4426950408889634f * kInvSqrtD);   // log2(e) / sqrt(D) * scale_q
 
-        // Sv: power of two >= every V scale of the key set.  P = p * scale_v / Sv
-        // stays <= 2^8 in f16; dividing p by Sv is folded into the exponent
-        // (log2 Sv is an integer), so the row sum and O carry the same 1/Sv
-        // factor and O / l needs no correction.
-        float vmax = 0.f;
-        for (int f = lane; f < p.n_frames_keys; f += 32)
-            vmax = fmaxf(vmax, __uint_as_float((uint32_t)(
-                                   p.v_scale_max[(size_t)p.slot[f] * H + h] & 0xffffffffull)));
+            // Sv: power of two >= every V scale of the key set
+            float vmax = 0.f;
+            for (int f = lane; f < p.n_frames_keys; f += 32)
+                vmax = fmaxf(vmax, __uint_as_float((uint32_t)(
+                                       p.v_scale_max[(size_t)p.slot[f] * H + h] & 0xffffffffull)));
 #pragma unroll
-        for (int o = 16; o >= 1; o >>= 1) vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, o));
-        int ve = (int)((__float_as_uint(vmax) >> 23) & 0xff);
-        if (__float_as_uint(vmax) & 0x7fffff) ve += 1;
-        if (!(vmax > 0.f)) ve = 127;
-        ve = max(127 - 60, min(127 + 60, ve));
-        const float log2_sv = (float)(ve - 127);
+            for (int o = 16; o >= 1; o >>= 1) vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, o));
+            int ve = (int)((__float_as_uint(vmax) >> 23) & 0xff);
+            if (__float_as_uint(vmax) & 0x7fffff) ve += 1;
+            if (!(vmax > 0.f)) ve = 127;
+            ve = max(127 - 60, min(127 + 60, ve));
+            const float log2_sv = (float)(ve - 127);
 
-        float m = -INFINITY;   // running max of s * scale_k (lazy)
-        float l = 0.f;         // running sum of p / Sv
-        const uint64_t c2c2 = pack2(c2, c2);
-        for (int j = 0; j < n_tiles && !fail; ++j) {
-            const int b = j & 1, st = j % kStages;
-            const int fi = j / p.tiles_per_frame;
-            const int nv = min(kBN, p.T - (j - fi * p.tiles_per_frame) * kBN);
-            if (!warp_wait(&sm.k_full[st], (j / kStages) & 1, limit)) { fail = true; break; }
-            if (!warp_wait(&sm.s_full[b], (j >> 1) & 1, limit)) { fail = true; break; }
-            tc_fence_after();
-            const uint32_t t_s = tmem + lane_off + (b ? kColS1 : kColS0);
-            // pass 1: row max over the valid keys
-            const float mt = nv == kBN ? tile_row_max<false>(t_s, sm.sk[st], nv)
-                                       : tile_row_max<true>(t_s, sm.sk[st], nv);
-            const float m_new = fmaxf(m, mt);
-            if (j == 0) {
-                m = m_new;   // first tile: O not yet written
-            } else if (__any_sync(0xffffffffu, (m_new - m) * c2 > kLazyRescaleLog2)) {
-                // Warp-uniform decision: the wait and the TMEM load/store below
-                // are warp-collective.  Every lane moves to its own new max
-                // (alpha = 1 where it did not grow).
-                const float alpha = ex2((m - m_new) * c2);
-                l *= alpha;
-                m = m_new;
-                // O holds PV up to tile j-1: wait for it, scale in place
-                if (!warp_wait(&sm.pv_done[(j - 1) & 1], ((j - 1) >> 1) & 1, limit)) { fail = true; break; }
+            float m = -INFINITY;   // running max of s * scale_k (lazy)
+            float l = 0.f;         // running sum of p / Sv
+            const uint64_t c2c2 = pack2(c2, c2);
+            for (int j = 0; j < n_tiles && !fail; ++j) {
+                const int st = j % kStages;
+                const int fi = j / p.tiles_per_frame;
+                const int nv = min(kBN, p.T - (j - fi * p.tiles_per_frame) * kBN);
+                if (!warp_wait(&sm.k_full[st], (j / kStages) & 1, limit)) { fail = true; break; }
+                if (!warp_wait(&sm.s_full[t], j & 1, limit)) { fail = true; break; }
                 tc_fence_after();
-                const uint32_t t_o = tmem + lane_off + kColO;
+                // pass 1: row max over the valid keys
+                const float mt = nv == kBN ? tile_row_max<false>(t_s, sm.sk[st], nv)
+                                           : tile_row_max<true>(t_s, sm.sk[st], nv);
+                const float m_new = fmaxf(m, mt);
+                if (j == 0) {
+                    m = m_new;   // first tile: O not yet written
+                } else if (__any_sync(0xffffffffu, (m_new - m) * c2 > kLazyRescaleLog2)) {
+                    // Warp-uniform decision (the TMEM load/store below are
+                    // warp-collective); every lane moves to its own new max
+                    // (alpha = 1 where it did not grow).  PV_t(j-1) completed
+                    // before S_t(j) was computed, so O_t is not being written.
+                    const float alpha = ex2((m - m_new) * c2);
+                    l *= alpha;
+                    m = m_new;
+#pragma unroll 1
+                    for (int c = 0; c < D / 32; ++c) {
+                        uint32_t o[32];
+                        tmem_ld32(t_o + c * 32, o);
+                        tc_wait_ld();
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+                        tmem_st32(t_o + c * 32, o);
+                    }
+                }
+                // pass 2: p / Sv = 2^(u*c2 - m*c2 - log2 Sv); P = (p / Sv) * scale_v
+                const float neg = -(m * c2 + log2_sv);
+                const uint64_t neg2 = pack2(neg, neg);
+                l += nv == kBN ? tile_make_p<false>(t_s, sm.sk[st], sm.sv[st], c2c2, neg2, nv)
+                               : tile_make_p<true>(t_s, sm.sk[st], sm.sv[st], c2c2, neg2, nv);
+                tc_wait_st();
+                tc_fence_before();
+                mbar_arrive(&sm.p_ready[t]);
+            }
+            if (!fail && !warp_wait(&sm.pv_done[t], (n_tiles - 1) & 1, limit)) fail = true;
+            if (!fail) {
+                tc_fence_after();
+                const float norm = 1.f / l;
 #pragma unroll 1
                 for (int c = 0; c < D / 32; ++c) {
                     uint32_t o[32];
                     tmem_ld32(t_o + c * 32, o);
                     tc_wait_ld();
+                    if (row_ok) {
+                        if (p.out_bf16) {
+                            __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(p.out) +
+                                                 ((size_t)qrow * H + h) * D + c * 32;
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-                    tmem_st32(t_o + c * 32, o);
-                }
-                tc_wait_st();
-            }
-            // P buffer b is free once PV(j-2) has completed
-            if (j >= 2 && !warp_wait(&sm.pv_done[b], ((j >> 1) - 1) & 1, limit)) { fail = true; break; }
-            tc_fence_after();
-
-            // pass 2: p / Sv = 2^(u*c2 - m*c2 - log2 Sv); P = (p / Sv) * scale_v
-            // in f16 into TMEM, 64 keys (32 columns) at a time
-            const float neg = -(m * c2 + log2_sv);
-            const uint64_t neg2 = pack2(neg, neg);
-            const uint32_t t_p = tmem + lane_off + (b ? kColP1 : kColP0);
-            l += nv == kBN ? tile_make_p<false>(t_s, t_p, sm.sk[st], sm.sv[st], c2c2, neg2, nv)
-                           : tile_make_p<true>(t_s, t_p, sm.sk[st], sm.sv[st], c2c2, neg2, nv);
-            tc_wait_st();
-            tc_fence_before();
-            mbar_arrive(&sm.s_free[b]);
-            mbar_arrive(&sm.p_ready[b]);
-        }
-        if (!fail && !warp_wait(&sm.o_done, 0, limit)) fail = true;
-        if (!fail) {
-            tc_fence_after();
-            const uint32_t t_o = tmem + lane_off + kColO;
-            const float norm = 1.f / l;
+                            for (int i = 0; i < 32; i += 8) {
+                                uint32_t w[4];
 #pragma unroll
-            for (int c = 0; c < D / 32; ++c) {
-                uint32_t o[32];
-                tmem_ld32(t_o + c * 32, o);
-                tc_wait_ld();
-                if (row_ok) {
-                    if (p.out_bf16) {
-                        __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(p.out) +
-                                             ((size_t)qrow * H + h) * D + c * 32;
+                                for (int e = 0; e < 4; ++e) {
+                                    __nv_bfloat162 a2 = __floats2bfloat162_rn(
+                                        __uint_as_float(o[i + 2 * e]) * norm,
+                                        __uint_as_float(o[i + 2 * e + 1]) * norm);
+                                    w[e] = *reinterpret_cast<uint32_t*>(&a2);
+                                }
+                                *reinterpret_cast<uint4*>(dst + i) = make_uint4(w[0], w[1], w[2], w[3]);
+                            }
+                        } else {
+                            float* dst = reinterpret_cast<float*>(p.out) + ((size_t)qrow * H + h) * D + c * 32;
 #pragma unroll
-                        for (int i = 0; i < 32; i += 8) {
-                            uint4 w;
-                            __nv_bfloat162 a0 = __floats2bfloat162_rn(__uint_as_float(o[i]) * norm, __uint_as_float(o[i + 1]) * norm);
-                            __nv_bfloat162 a1 = __floats2bfloat162_rn(__uint_as_float(o[i + 2]) * norm, __uint_as_float(o[i + 3]) * norm);
-                            __nv_bfloat162 a2 = __floats2bfloat162_rn(__uint_as_float(o[i + 4]) * norm, __uint_as_float(o[i + 5]) * norm);
-                            __nv_bfloat162 a3 = __floats2bfloat162_rn(__uint_as_float(o[i + 6]) * norm, __uint_as_float(o[i + 7]) * norm);
-                            w.x = *reinterpret_cast<uint32_t*>(&a0);
-                            w.y = *reinterpret_cast<uint32_t*>(&a1);
-                            w.z = *reinterpret_cast<uint32_t*>(&a2);
-                            w.w = *reinterpret_cast<uint32_t*>(&a3);
-                            *reinterpret_cast<uint4*>(dst + i) = w;
+                            for (int i = 0; i < 32; i += 4)
+                                *reinterpret_cast<float4*>(dst + i) = make_float4(
+                                    __uint_as_float(o[i]) * norm, __uint_as_float(o[i + 1]) * norm,
+                                    __uint_as_float(o[i + 2]) * norm, __uint_as_float(o[i + 3]) * norm);
                         }
-                    } else {
-                        float* dst = reinterpret_cast<float*>(p.out) + ((size_t)qrow * H + h) * D + c * 32;
-#pragma unroll
-                        for (int i = 0; i < 32; i += 4)
-                            *reinterpret_cast<float4*>(dst + i) = make_float4(
-                                __uint_as_float(o[i]) * norm, __uint_as_float(o[i + 1]) * norm,
-                                __uint_as_float(o[i + 2]) * norm, __uint_as_float(o[i + 3]) * norm);
                     }
                 }
             }
         }
     }
 
-    if (fail) {
-        atomicOr(p.err, kErrTimeout);
-        sm.failed = 1;
-    }
+    if (fail) atomicOr(p.err, kErrTimeout);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -515,14 +536,16 @@ template <int D>
 cudaError_t launch(const AttendParams& p, const CUtensorMap* maps, cudaStream_t stream)
 {
     const size_t smem = sizeof(Smem<D>) + 1024;
-    static bool configured = false;
-    if (!configured) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    static unsigned configured = 0;   // bit per device
+    if (dev < 32 && !(configured & (1u << dev))) {
         cudaError_t e = cudaFuncSetAttribute(attend_kernel<D>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
-        configured = true;
+        configured |= 1u << dev;
     }
-    dim3 grid((p.M + kBM - 1) / kBM, p.H);
+    dim3 grid((p.M + kQT * kBM - 1) / (kQT * kBM), p.H);
     attend_kernel<D><<<grid, kThreads, smem, stream>>>(p, maps[0], maps[1], maps[2], maps[3], maps[4]);
     return cudaGetLastError();
 }
