@@ -13,16 +13,17 @@
 // loads; 12 warps:
 //   warp 0     TMA producer: both Q tiles once; per KV tile the K and V code
 //              tiles at (ring slot * H + head, token tile) and their scales.
-//   warp 1     TMEM owner and MMA issuer.  Per query tile t and KV tile j:
-//              S_t = Q_t K_j^T (kind::f8f6f4, E4M3 x E4M3 -> f32 in TMEM),
-//              then O_t += P_t V16_j (kind::f16, P_t read from TMEM where it
-//              overwrote S_t, V16 from shared memory).  It issues whichever of
-//              the two tiles' next MMAs is ready, so one tile's softmax runs
-//              while the other tile's MMAs are on the tensor core.
-//   warps 2-3  widen the V code tile to f16 (exact) in the MN-major layout
+//   warps 1,3  MMA issuers, one per query tile t (warp 1 also owns TMEM).  Per
+//              KV tile j: S_t = Q_t K_j^T (kind::f8f6f4, E4M3 x E4M3 -> f32 in
+//              TMEM), then O_t += P_t V16_j (kind::f16, P_t read from TMEM where
+//              it overwrote S_t, V16 from shared memory).  Two independent
+//              issuers let one tile's softmax run while the other tile's MMAs
+//              are on the tensor core, with blocking waits and no polling.
+//   warp 2     widens the V code tile to f16 (exact) in the MN-major layout
 //              the PV MMA reads.
 //   warps 4-7  softmax of query tile 0, warps 8-11 of query tile 1; one query
-//              row per thread: s*scale_k, running max, exp2, row sum,
+//              row per thread, the tile's 128 scores held in registers (one
+//              TMEM round trip per KV tile): s*scale_k, running max, exp2, row sum,
 //              P = p*scale_v/Sv in f16 written back over S; lazy O rescaling
 //              only when the running max grows by more than 2^8.
 // TMEM columns: S_0 [0,128), S_1 [128,256), O_0 [256,256+D), O_1 [384,384+D).
@@ -38,6 +39,10 @@
 // set (from the per-frame V-scale maxima the append kernel records); P =
 // p*scale_v/Sv stays <= 2^8 inside f16 range, and 1/Sv is folded into the
 // exponent so the row sum carries the same factor and O/l needs none.
+//
+// Registers: the block launches with 168 per thread; the four single-role
+// warps give theirs back (setmaxnreg 56) and the softmax warps take them
+// (setmaxnreg 224): 128 x 56 + 256 x 224 = 384 x 168.
 //
 // Every mbarrier wait is bounded; on time-out a thread sets the error word,
 // leaves its loop, and the CTA drains its own async work before returning.
@@ -79,7 +84,7 @@ struct Smem {
     uint64_t kv_empty[kStages];
     uint64_t s_full[kQT], p_ready[kQT], pv_done[kQT];
     uint64_t v16_ready[2], tile_done[2];
-    uint64_t drain;
+    uint64_t drain[kQT];
     uint32_t tmem_base;
 };
 
@@ -141,72 +146,68 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, long l
     return __all_sync(0xffffffffu, mbar_wait(bar, parity, limit));
 }
 
-// Pass 1 of a KV tile: row max of u = s * scale_k over the valid keys, S read
-// from TMEM in 32-column chunks.  kMask: tile with fewer than 128 valid keys.
+// Pass 1 of a KV tile, on the 128 scores of this thread's row held in
+// registers: u = s * scale_k (written back over s, in pairs) and the row max of
+// u over the valid keys.  kMask: tile with fewer than 128 valid keys.
 template <bool kMask>
-__device__ __forceinline__ float tile_row_max(uint32_t t_s, const float* sk, int nv)
+__device__ __forceinline__ float tile_row_max(uint32_t* sr, const float* sk, int nv)
 {
     const float4* sk4 = reinterpret_cast<const float4*>(sk);
     float mt0 = -INFINITY, mt1 = -INFINITY;
 #pragma unroll
-    for (int c = 0; c < kBN / 32; ++c) {
-        uint32_t sr[32];
-        tmem_ld32(t_s + c * 32, sr);
-        tc_wait_ld();
-#pragma unroll
-        for (int k4 = 0; k4 < 8; ++k4) {
-            const float4 kk = sk4[c * 8 + k4];
-            float a, b, cc, d;
-            unpack2(mul2(pack2(__uint_as_float(sr[4 * k4]), __uint_as_float(sr[4 * k4 + 1])),
-                         pack2(kk.x, kk.y)), a, b);
-            unpack2(mul2(pack2(__uint_as_float(sr[4 * k4 + 2]), __uint_as_float(sr[4 * k4 + 3])),
-                         pack2(kk.z, kk.w)), cc, d);
-            if (!kMask) {
-                mt0 = max3(mt0, a, b);
-                mt1 = max3(mt1, cc, d);
-            } else {
-                const int k = c * 32 + 4 * k4;
-                if (k < nv) mt0 = fmaxf(mt0, a);
-                if (k + 1 < nv) mt1 = fmaxf(mt1, b);
-                if (k + 2 < nv) mt0 = fmaxf(mt0, cc);
-                if (k + 3 < nv) mt1 = fmaxf(mt1, d);
-            }
+    for (int k4 = 0; k4 < kBN / 4; ++k4) {
+        // keep the scale loads to one 32-key chunk in flight (registers: the
+        // 128 scores already occupy most of the thread's budget)
+        if ((k4 & 7) == 0) asm volatile("" ::: "memory");
+        const float4 kk = sk4[k4];
+        const uint64_t u0 = mul2(pack2(__uint_as_float(sr[4 * k4]), __uint_as_float(sr[4 * k4 + 1])),
+                                 pack2(kk.x, kk.y));
+        const uint64_t u1 = mul2(pack2(__uint_as_float(sr[4 * k4 + 2]), __uint_as_float(sr[4 * k4 + 3])),
+                                 pack2(kk.z, kk.w));
+        float a, b, c, d;
+        unpack2(u0, a, b);
+        unpack2(u1, c, d);
+        sr[4 * k4] = __float_as_uint(a);
+        sr[4 * k4 + 1] = __float_as_uint(b);
+        sr[4 * k4 + 2] = __float_as_uint(c);
+        sr[4 * k4 + 3] = __float_as_uint(d);
+        if (!kMask) {
+            mt0 = max3(mt0, a, b);
+            mt1 = max3(mt1, c, d);
+        } else {
+            const int k = 4 * k4;
+            if (k < nv) mt0 = fmaxf(mt0, a);
+            if (k + 1 < nv) mt1 = fmaxf(mt1, b);
+            if (k + 2 < nv) mt0 = fmaxf(mt0, c);
+            if (k + 3 < nv) mt1 = fmaxf(mt1, d);
         }
     }
     return fmaxf(mt0, mt1);
 }
 
 // Pass 2 of a KV tile: p/Sv = 2^(u*c2 + neg), P = (p/Sv) * scale_v packed to
-// f16 pairs and written over S in TMEM: the 32 keys of S columns [32c, 32c+32)
-// become P columns [16c, 16c+16), which were all read before (in this chunk or
-// the previous one).  Returns the tile's row sum of p/Sv.
+// f16 pairs and written over S in TMEM (keys [32c, 32c+32) -> P columns
+// [16c, 16c+16); all of S was read before).  Returns the row sum of p/Sv.
 template <bool kMask>
-__device__ __forceinline__ float tile_make_p(uint32_t t_s, const float* sk, const float* sv,
+__device__ __forceinline__ float tile_make_p(const uint32_t* sr, uint32_t t_s, const float* sv,
                                              uint64_t c2c2, uint64_t neg2, int nv)
 {
-    const float4* sk4 = reinterpret_cast<const float4*>(sk);
     const float4* sv4 = reinterpret_cast<const float4*>(sv);
     uint64_t ls2 = pack2(0.f, 0.f);
 #pragma unroll
     for (int c = 0; c < kBN / 32; ++c) {
-        uint32_t sr[32];
-        tmem_ld32(t_s + c * 32, sr);
-        tc_wait_ld();
         uint32_t pk[16];
 #pragma unroll
         for (int k4 = 0; k4 < 8; ++k4) {
-            const float4 kk = sk4[c * 8 + k4];
             const float4 vv = sv4[c * 8 + k4];
 #pragma unroll
             for (int hh = 0; hh < 2; ++hh) {
-                const int kl = 4 * k4 + 2 * hh;
-                const uint64_t u = mul2(pack2(__uint_as_float(sr[kl]), __uint_as_float(sr[kl + 1])),
-                                        hh ? pack2(kk.z, kk.w) : pack2(kk.x, kk.y));
+                const int k = c * 32 + 4 * k4 + 2 * hh;
                 float x0, x1;
-                unpack2(fma2(u, c2c2, neg2), x0, x1);
+                unpack2(fma2(pack2(__uint_as_float(sr[k]), __uint_as_float(sr[k + 1])), c2c2, neg2),
+                        x0, x1);
                 float p0 = ex2(x0), p1 = ex2(x1);
                 if (kMask) {
-                    const int k = c * 32 + kl;
                     if (k >= nv) p0 = 0.f;
                     if (k + 1 >= nv) p1 = 0.f;
                 }
@@ -215,7 +216,7 @@ __device__ __forceinline__ float tile_make_p(uint32_t t_s, const float* sk, cons
                 float q0, q1;
                 unpack2(mul2(pp, hh ? pack2(vv.z, vv.w) : pack2(vv.x, vv.y)), q0, q1);
                 __half2 hv = __floats2half2_rn(q0, q1);
-                pk[kl / 2] = *reinterpret_cast<uint32_t*>(&hv);
+                pk[(4 * k4 + 2 * hh) / 2] = *reinterpret_cast<uint32_t*>(&hv);
             }
         }
         tmem_st16(t_s + c * 16, pk);
@@ -224,6 +225,9 @@ __device__ __forceinline__ float tile_make_p(uint32_t t_s, const float* sk, cons
     unpack2(ls2, a, b);
     return a + b;
 }
+
+__device__ __forceinline__ void reg_dealloc_56() { asm volatile("setmaxnreg.dec.sync.aligned.u32 56;"); }
+__device__ __forceinline__ void reg_alloc_224() { asm volatile("setmaxnreg.inc.sync.aligned.u32 224;"); }
 
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -248,20 +252,21 @@ attend_kernel(const __grid_constant__ AttendParams p, const __grid_constant__ CU
 
     if (threadIdx.x == 0) {
         mbar_init(&sm.q_full, 1);
+        // kv_empty / tile_done: one commit from each active query tile's issuer
         for (int s = 0; s < kStages; ++s) {
             mbar_init(&sm.k_full[s], 1);
-            mbar_init(&sm.kv_empty[s], 1);
+            mbar_init(&sm.kv_empty[s], n_qt);
         }
         for (int t = 0; t < kQT; ++t) {
             mbar_init(&sm.s_full[t], 1);
             mbar_init(&sm.p_ready[t], 128);
             mbar_init(&sm.pv_done[t], 1);
+            mbar_init(&sm.drain[t], 1);
         }
         for (int b = 0; b < 2; ++b) {
-            mbar_init(&sm.v16_ready[b], 64);
-            mbar_init(&sm.tile_done[b], 1);
+            mbar_init(&sm.v16_ready[b], 32);
+            mbar_init(&sm.tile_done[b], n_qt);
         }
-        mbar_init(&sm.drain, 1);
         fence_mbar_init();
     }
     if (warp == 1) {
@@ -281,140 +286,122 @@ attend_kernel(const __grid_constant__ AttendParams p, const __grid_constant__ CU
     const uint32_t tmem = sm.tmem_base;
     bool fail = false;
 
-    if (warp == 0) {
-        // ------------------------------------------------------ producer --
-        if (lane == 0 && !p.debug_wait_fault) {
-            constexpr uint32_t kTileBytes = Smem<D>::kTileBytes;
-            mbar_arrive_expect_tx(&sm.q_full, kQT * kTileBytes);
-            for (int t = 0; t < kQT; ++t) tma_load_3d(sm.q[t], &map_q, &sm.q_full, 0, q0 + t * kBM, h);
-            int issued = 0;
-            for (int j = 0; j < n_tiles; ++j) {
-                const int st = j % kStages;
-                if (j >= kStages &&
-                    !mbar_wait(&sm.kv_empty[st], ((j / kStages) - 1) & 1, limit)) {
-                    fail = true;
-                    break;
-                }
-                const int fi = j / p.tiles_per_frame;
-                const int t0 = (j - fi * p.tiles_per_frame) * kBN;
-                const int row = p.slot[fi] * H + h;
-                mbar_arrive_expect_tx(&sm.k_full[st], 2 * kTileBytes + 2 * kBN * 4);
-                tma_load_3d(sm.k[st], &map_k, &sm.k_full[st], 0, t0, row);
-                tma_load_3d(sm.v8[st], &map_v, &sm.k_full[st], 0, t0, row);
-                tma_load_2d(sm.sk[st], &map_sk, &sm.k_full[st], t0, row);
-                tma_load_2d(sm.sv[st], &map_sv, &sm.k_full[st], t0, row);
-                ++issued;
-            }
-            // drain: every copy this thread issued has landed before the CTA may exit
-            mbar_wait(&sm.q_full, 0, limit);
-            for (int j = issued - kStages; j < issued; ++j) {
-                if (j < 0) continue;
-                mbar_wait(&sm.k_full[j % kStages], (j / kStages) & 1, limit);
-            }
-        }
-    } else if (warp == 1) {
-        // ---------------------------------------------------- MMA issuer --
-        if (lane == 0) {
-            constexpr uint32_t kQK = idesc(kBM, kBN, 0, 0, 0, 0);        // E4M3 x E4M3 -> f32
-            constexpr uint32_t kPV = idesc(kBM, D, 0, 0, 0, 1);          // f16 x f16(MN) -> f32
-            constexpr uint32_t kSw = D == 128 ? kSwizzle128 : kSwizzle64;
-            constexpr uint32_t kSbo = D == 128 ? 1024 : 512;
-            int qk_next[kQT] = {0, 0}, pv_next[kQT] = {0, 0};
-            if (!mbar_wait(&sm.q_full, 0, limit)) fail = true;
-            long long last = clock64();
-            while (!fail) {
-                bool done = true, progressed = false;
-                for (int t = 0; t < n_qt; ++t) {
-                    if (pv_next[t] < n_tiles) done = false;
-                    // S_t = Q_t K_j^T once K_j has landed and PV_t(j-1) has completed
-                    int j = qk_next[t];
-                    if (j < n_tiles && j == pv_next[t] &&
-                        mbar_test(&sm.k_full[j % kStages], (j / kStages) & 1) &&
-                        (j == 0 || mbar_test(&sm.pv_done[t], (j - 1) & 1))) {
-                        tc_fence_after();
-                        const uint32_t q_addr = smem_u32(sm.q[t]);
-                        const uint32_t k_addr = smem_u32(sm.k[j % kStages]);
-#pragma unroll
-                        for (int kk = 0; kk < D / 32; ++kk)
-                            mma_f8_ss(tmem + col_s(t), smem_desc(q_addr + kk * 32, 16, kSbo, kSw),
-                                      smem_desc(k_addr + kk * 32, 16, kSbo, kSw), kQK, kk > 0);
-                        tc_commit(&sm.s_full[t]);
-                        qk_next[t] = j + 1;
-                        progressed = true;
+    // setmaxnreg is executed by whole warpgroups (warps 0-3, 4-7, 8-11), as the
+    // first instruction of each warpgroup's branch, so every region is
+    // allocated by ptxas under the budget it runs with.
+    if (warp < 4) {
+        reg_dealloc_56();
+        if (warp == 0) {
+            // ------------------------------------------------------ producer --
+            if (lane == 0 && !p.debug_wait_fault) {
+                constexpr uint32_t kTileBytes = Smem<D>::kTileBytes;
+                mbar_arrive_expect_tx(&sm.q_full, kQT * kTileBytes);
+                for (int t = 0; t < kQT; ++t) tma_load_3d(sm.q[t], &map_q, &sm.q_full, 0, q0 + t * kBM, h);
+                int issued = 0;
+                for (int j = 0; j < n_tiles; ++j) {
+                    const int st = j % kStages;
+                    if (j >= kStages &&
+                        !mbar_wait(&sm.kv_empty[st], ((j / kStages) - 1) & 1, limit)) {
+                        fail = true;
+                        break;
                     }
+                    const int fi = j / p.tiles_per_frame;
+                    const int t0 = (j - fi * p.tiles_per_frame) * kBN;
+                    const int row = p.slot[fi] * H + h;
+                    mbar_arrive_expect_tx(&sm.k_full[st], 2 * kTileBytes + 2 * kBN * 4);
+                    tma_load_3d(sm.k[st], &map_k, &sm.k_full[st], 0, t0, row);
+                    tma_load_3d(sm.v8[st], &map_v, &sm.k_full[st], 0, t0, row);
+                    tma_load_2d(sm.sk[st], &map_sk, &sm.k_full[st], t0, row);
+                    tma_load_2d(sm.sv[st], &map_sv, &sm.k_full[st], t0, row);
+                    ++issued;
+                }
+                // drain: every copy this thread issued has landed before the CTA may exit
+                mbar_wait(&sm.q_full, 0, limit);
+                for (int j = issued - kStages; j < issued; ++j) {
+                    if (j < 0) continue;
+                    mbar_wait(&sm.k_full[j % kStages], (j / kStages) & 1, limit);
+                }
+            }
+        } else if (warp == 1 || warp == 3) {
+            // ------------------------------------- MMA issuer of query tile t --
+            const int t = warp == 1 ? 0 : 1;
+            if (lane == 0 && t < n_qt) {
+                constexpr uint32_t kQK = idesc(kBM, kBN, 0, 0, 0, 0);        // E4M3 x E4M3 -> f32
+                constexpr uint32_t kPV = idesc(kBM, D, 0, 0, 0, 1);          // f16 x f16(MN) -> f32
+                constexpr uint32_t kSw = D == 128 ? kSwizzle128 : kSwizzle64;
+                constexpr uint32_t kSbo = D == 128 ? 1024 : 512;
+                const uint32_t q_addr = smem_u32(sm.q[t]);
+                if (!mbar_wait(&sm.q_full, 0, limit)) fail = true;
+                for (int j = 0; j < n_tiles && !fail; ++j) {
+                    // S_t = Q_t K_j^T once K_j has landed and PV_t(j-1) (which reads
+                    // P_t out of the S_t columns) has completed
+                    if (!mbar_wait(&sm.k_full[j % kStages], (j / kStages) & 1, limit)) { fail = true; break; }
+                    if (j > 0 && !mbar_wait(&sm.pv_done[t], (j - 1) & 1, limit)) { fail = true; break; }
+                    tc_fence_after();
+                    const uint32_t k_addr = smem_u32(sm.k[j % kStages]);
+    #pragma unroll
+                    for (int kk = 0; kk < D / 32; ++kk)
+                        mma_f8_ss(tmem + col_s(t), smem_desc(q_addr + kk * 32, 16, kSbo, kSw),
+                                  smem_desc(k_addr + kk * 32, 16, kSbo, kSw), kQK, kk > 0);
+                    tc_commit(&sm.s_full[t]);
                     // O_t += P_t V_j once the softmax wrote P_t and V_j is widened
-                    j = pv_next[t];
-                    if (j < qk_next[t] && mbar_test(&sm.p_ready[t], j & 1) &&
-                        mbar_test(&sm.v16_ready[j & 1], (j >> 1) & 1)) {
-                        tc_fence_after();
-                        const uint32_t v_addr = smem_u32(sm.v16[j & 1]);
-#pragma unroll
-                        for (int kk = 0; kk < kBN / 16; ++kk)
-                            mma_f16_ts(tmem + col_o(t), tmem + col_s(t) + kk * 8,
-                                       smem_desc(v_addr + kk * 2048, 16384, 1024, kSwizzle128), kPV,
-                                       (j > 0 || kk > 0) ? 1u : 0u);
-                        tc_commit(&sm.pv_done[t]);
-                        pv_next[t] = j + 1;
-                        progressed = true;
-                        bool all = true;
-                        for (int u = 0; u < n_qt; ++u) all &= pv_next[u] > j;
-                        if (all) {   // every query tile consumed KV tile j
-                            tc_commit(&sm.kv_empty[j % kStages]);
-                            tc_commit(&sm.tile_done[j & 1]);
-                        }
-                    }
+                    if (!mbar_wait(&sm.p_ready[t], j & 1, limit)) { fail = true; break; }
+                    if (!mbar_wait(&sm.v16_ready[j & 1], (j >> 1) & 1, limit)) { fail = true; break; }
+                    tc_fence_after();
+                    const uint32_t v_addr = smem_u32(sm.v16[j & 1]);
+    #pragma unroll
+                    for (int kk = 0; kk < kBN / 16; ++kk)
+                        mma_f16_ts(tmem + col_o(t), tmem + col_s(t) + kk * 8,
+                                   smem_desc(v_addr + kk * 2048, 16384, 1024, kSwizzle128), kPV,
+                                   (j > 0 || kk > 0) ? 1u : 0u);
+                    tc_commit(&sm.pv_done[t]);
+                    tc_commit(&sm.kv_empty[j % kStages]);
+                    tc_commit(&sm.tile_done[j & 1]);
                 }
-                if (done) break;
-                if (progressed) {
-                    last = clock64();
-                } else {
-                    if (clock64() - last > limit) fail = true;
-                    __nanosleep(20);
+                // drain: all MMAs issued by this thread complete before TMEM is freed
+                tc_commit(&sm.drain[t]);
+                if (!mbar_wait(&sm.drain[t], 0, limit)) fail = true;
+            }
+        } else if (warp == 2) {
+            // ------------------------------------------- V widening (FP8->f16) --
+            // A warp step covers 8 consecutive key rows x 4 chunk columns of one
+            // 64-element block: in every 8-lane shared-memory phase the 8 rows hit
+            // 8 different 16-byte bank groups, for the swizzled reads and for both
+            // swizzled writes.
+            constexpr int kNB = D / 64;                 // 64-element blocks per key row
+            const int rl = lane & 7, cq = lane >> 3;
+            for (int j = 0; j < n_tiles; ++j) {
+                const int st = j % kStages, b = j & 1;
+                if (!warp_wait(&sm.k_full[st], (j / kStages) & 1, limit)) { fail = true; break; }
+                if (j >= 2 && !warp_wait(&sm.tile_done[b], ((j >> 1) - 1) & 1, limit)) { fail = true; break; }
+                const uint8_t* src = sm.v8[st];
+                uint8_t* dst = sm.v16[b];
+    #pragma unroll 4
+                for (int combo = 0; combo < (kBN / 8) * kNB; ++combo) {
+                    const int r = (combo / kNB) * 8 + rl;
+                    const int nb = combo % kNB;
+                    const int c = nb * 4 + cq;                              // 16-byte chunk of the FP8 row
+                    const int sc = D == 128 ? (c ^ (r & 7)) : (c ^ ((r >> 1) & 3));
+                    const uint4 raw = *reinterpret_cast<const uint4*>(src + r * D + sc * 16);
+                    uint32_t o[8];
+                    e4m3x4_to_f16x4(raw.x, o[0], o[1]);
+                    e4m3x4_to_f16x4(raw.y, o[2], o[3]);
+                    e4m3x4_to_f16x4(raw.z, o[4], o[5]);
+                    e4m3x4_to_f16x4(raw.w, o[6], o[7]);
+                    // elements d = 16c .. 16c+15 = block nb, bytes 32*cq .. 32*cq+31 of the row
+                    uint8_t* rowp = dst + nb * (kBN * 128) + r * 128;
+                    *reinterpret_cast<uint4*>(rowp + (((2 * cq) ^ (r & 7)) << 4)) =
+                        make_uint4(o[0], o[1], o[2], o[3]);
+                    *reinterpret_cast<uint4*>(rowp + (((2 * cq + 1) ^ (r & 7)) << 4)) =
+                        make_uint4(o[4], o[5], o[6], o[7]);
                 }
+                fence_async_smem();   // generic-proxy writes -> visible to the MMA's async proxy
+                mbar_arrive(&sm.v16_ready[b]);
             }
-            // drain: all MMAs issued by this thread complete before TMEM is freed
-            tc_commit(&sm.drain);
-            if (!mbar_wait(&sm.drain, 0, limit)) fail = true;
-        }
-    } else if (warp < 4) {
-        // ------------------------------------------- V widening (FP8->f16) --
-        // A warp step covers 8 consecutive key rows x 4 chunk columns of one
-        // 64-element block: in every 8-lane shared-memory phase the 8 rows hit
-        // 8 different 16-byte bank groups, for the swizzled reads and for both
-        // swizzled writes.
-        constexpr int kNB = D / 64;                 // 64-element blocks per key row
-        const int wv = warp - 2;                    // converter warp 0/1
-        const int rl = lane & 7, cq = lane >> 3;
-        for (int j = 0; j < n_tiles; ++j) {
-            const int st = j % kStages, b = j & 1;
-            if (!warp_wait(&sm.k_full[st], (j / kStages) & 1, limit)) { fail = true; break; }
-            if (j >= 2 && !warp_wait(&sm.tile_done[b], ((j >> 1) - 1) & 1, limit)) { fail = true; break; }
-            const uint8_t* src = sm.v8[st];
-            uint8_t* dst = sm.v16[b];
-#pragma unroll 4
-            for (int combo = wv; combo < (kBN / 8) * kNB; combo += 2) {
-                const int r = (combo / kNB) * 8 + rl;
-                const int nb = combo % kNB;
-                const int c = nb * 4 + cq;                              // 16-byte chunk of the FP8 row
-                const int sc = D == 128 ? (c ^ (r & 7)) : (c ^ ((r >> 1) & 3));
-                const uint4 raw = *reinterpret_cast<const uint4*>(src + r * D + sc * 16);
-                uint32_t o[8];
-                e4m3x4_to_f16x4(raw.x, o[0], o[1]);
-                e4m3x4_to_f16x4(raw.y, o[2], o[3]);
-                e4m3x4_to_f16x4(raw.z, o[4], o[5]);
-                e4m3x4_to_f16x4(raw.w, o[6], o[7]);
-                // elements d = 16c .. 16c+15 = block nb, bytes 32*cq .. 32*cq+31 of the row
-                uint8_t* rowp = dst + nb * (kBN * 128) + r * 128;
-                *reinterpret_cast<uint4*>(rowp + (((2 * cq) ^ (r & 7)) << 4)) =
-                    make_uint4(o[0], o[1], o[2], o[3]);
-                *reinterpret_cast<uint4*>(rowp + (((2 * cq + 1) ^ (r & 7)) << 4)) =
-                    make_uint4(o[4], o[5], o[6], o[7]);
-            }
-            fence_async_smem();   // generic-proxy writes -> visible to the MMA's async proxy
-            mbar_arrive(&sm.v16_ready[b]);
         }
     } else {
         // --------------------------------------------------------- softmax --
+        reg_alloc_224();
         const int t = (warp - 4) >> 2;              // query tile of this warpgroup
         if (t < n_qt) {
             const int row = (warp & 3) * 32 + lane;     // TMEM lane == query row in tile
@@ -450,9 +437,13 @@ attend_kernel(const __grid_constant__ AttendParams p, const __grid_constant__ CU
                 if (!warp_wait(&sm.k_full[st], (j / kStages) & 1, limit)) { fail = true; break; }
                 if (!warp_wait(&sm.s_full[t], j & 1, limit)) { fail = true; break; }
                 tc_fence_after();
-                // pass 1: row max over the valid keys
-                const float mt = nv == kBN ? tile_row_max<false>(t_s, sm.sk[st], nv)
-                                           : tile_row_max<true>(t_s, sm.sk[st], nv);
+                uint32_t sr[kBN];
+#pragma unroll
+                for (int c = 0; c < kBN / 32; ++c) tmem_ld32(t_s + c * 32, sr + c * 32);
+                tc_wait_ld();
+                // pass 1: u = s * scale_k and the row max over the valid keys
+                const float mt = nv == kBN ? tile_row_max<false>(sr, sm.sk[st], nv)
+                                           : tile_row_max<true>(sr, sm.sk[st], nv);
                 const float m_new = fmaxf(m, mt);
                 if (j == 0) {
                     m = m_new;   // first tile: O not yet written
@@ -477,8 +468,8 @@ attend_kernel(const __grid_constant__ AttendParams p, const __grid_constant__ CU
                 // pass 2: p / Sv = 2^(u*c2 - m*c2 - log2 Sv); P = (p / Sv) * scale_v
                 const float neg = -(m * c2 + log2_sv);
                 const uint64_t neg2 = pack2(neg, neg);
-                l += nv == kBN ? tile_make_p<false>(t_s, sm.sk[st], sm.sv[st], c2c2, neg2, nv)
-                               : tile_make_p<true>(t_s, sm.sk[st], sm.sv[st], c2c2, neg2, nv);
+                l += nv == kBN ? tile_make_p<false>(sr, t_s, sm.sv[st], c2c2, neg2, nv)
+                               : tile_make_p<true>(sr, t_s, sm.sv[st], c2c2, neg2, nv);
                 tc_wait_st();
                 tc_fence_before();
                 mbar_arrive(&sm.p_ready[t]);
