@@ -85,6 +85,7 @@ struct Smem {
     uint64_t s_full[kQT], p_ready[kQT], pv_done[kQT];
     uint64_t v16_ready[2], tile_done[2];
     uint64_t drain[kQT];
+    uint64_t exp_turn[kQT];   // alternation of the two softmax warpgroups' exp phases
     uint32_t tmem_base;
 };
 
@@ -144,6 +145,10 @@ __device__ __forceinline__ void e4m3x4_to_f16x4(uint32_t w, uint32_t& lo, uint32
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, long long limit)
 {
     return __all_sync(0xffffffffu, mbar_wait(bar, parity, limit));
+}
+__device__ __forceinline__ bool warp_wait_sleep(uint64_t* bar, uint32_t parity, long long limit)
+{
+    return __all_sync(0xffffffffu, mbar_wait_sleep(bar, parity, limit));
 }
 
 // Pass 1 of a KV tile, on the 128 scores of this thread's row held in
@@ -262,6 +267,7 @@ attend_kernel(const __grid_constant__ AttendParams p, const __grid_constant__ CU
             mbar_init(&sm.p_ready[t], 128);
             mbar_init(&sm.pv_done[t], 1);
             mbar_init(&sm.drain[t], 1);
+            mbar_init(&sm.exp_turn[t], 128);
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&sm.v16_ready[b], 32);
@@ -301,7 +307,7 @@ attend_kernel(const __grid_constant__ AttendParams p, const __grid_constant__ CU
                 for (int j = 0; j < n_tiles; ++j) {
                     const int st = j % kStages;
                     if (j >= kStages &&
-                        !mbar_wait(&sm.kv_empty[st], ((j / kStages) - 1) & 1, limit)) {
+                        !mbar_wait_sleep(&sm.kv_empty[st], ((j / kStages) - 1) & 1, limit)) {
                         fail = true;
                         break;
                     }
@@ -372,8 +378,8 @@ attend_kernel(const __grid_constant__ AttendParams p, const __grid_constant__ CU
             const int rl = lane & 7, cq = lane >> 3;
             for (int j = 0; j < n_tiles; ++j) {
                 const int st = j % kStages, b = j & 1;
-                if (!warp_wait(&sm.k_full[st], (j / kStages) & 1, limit)) { fail = true; break; }
-                if (j >= 2 && !warp_wait(&sm.tile_done[b], ((j >> 1) - 1) & 1, limit)) { fail = true; break; }
+                if (!warp_wait_sleep(&sm.k_full[st], (j / kStages) & 1, limit)) { fail = true; break; }
+                if (j >= 2 && !warp_wait_sleep(&sm.tile_done[b], ((j >> 1) - 1) & 1, limit)) { fail = true; break; }
                 const uint8_t* src = sm.v8[st];
                 uint8_t* dst = sm.v16[b];
     #pragma unroll 4
@@ -465,11 +471,19 @@ attend_kernel(const __grid_constant__ AttendParams p, const __grid_constant__ CU
                         tmem_st32(t_o + c * 32, o);
                     }
                 }
-                // pass 2: p / Sv = 2^(u*c2 - m*c2 - log2 Sv); P = (p / Sv) * scale_v
+                // pass 2: p / Sv = 2^(u*c2 - m*c2 - log2 Sv); P = (p / Sv) * scale_v.
+                // With two query tiles the warpgroups take turns (tile 0 of
+                // KV tile j, tile 1 of j, tile 0 of j+1, ...): each exp phase
+                // then runs with the exp unit to itself, and one tile's PV and
+                // next QK overlap the other tile's exp phase.
+                const bool pingpong = n_qt == 2;
+                if (pingpong && (t == 1 || j > 0) &&
+                    !warp_wait(&sm.exp_turn[t], (t == 1 ? j : j - 1) & 1, limit)) { fail = true; break; }
                 const float neg = -(m * c2 + log2_sv);
                 const uint64_t neg2 = pack2(neg, neg);
                 l += nv == kBN ? tile_make_p<false>(sr, t_s, sm.sv[st], c2c2, neg2, nv)
                                : tile_make_p<true>(sr, t_s, sm.sv[st], c2c2, neg2, nv);
+                if (pingpong) mbar_arrive(&sm.exp_turn[1 - t]);
                 tc_wait_st();
                 tc_fence_before();
                 mbar_arrive(&sm.p_ready[t]);

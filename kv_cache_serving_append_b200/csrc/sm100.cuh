@@ -39,17 +39,31 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
         "r"(bytes)
         : "memory");
 }
-// try_wait with a suspend-time hint: a thread whose phase is not complete is
-// suspended in hardware (up to the hint, in ns) instead of spinning, so
-// waiting warps do not take issue slots from the warps doing the math.
+// try_wait: returns when the phase completes or after a short hardware time
+// limit.  Spinning on it keeps the wake-up latency of a critical-path wait to
+// tens of cycles.
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+// try_wait with a suspend-time hint (ns): the thread is suspended in hardware
+// instead of spinning -- for waits off the critical path, where the slower
+// wake-up does not matter but the freed issue slots do.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity)
 {
     uint32_t ok;
     asm volatile(
         "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity), "r"(1000000u)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(100000u)
         : "memory");
     return ok != 0;
 }
@@ -65,12 +79,21 @@ __device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity)
         : "memory");
     return ok != 0;
 }
-// Bounded wait: returns false when the limit (in SM clock cycles) runs out.
+// Bounded waits: return false when the limit (in SM clock cycles) runs out.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, long long limit)
 {
     if (mbar_try_wait(bar, parity)) return true;
     const long long t0 = clock64();
     while (!mbar_try_wait(bar, parity)) {
+        if (clock64() - t0 > limit) return false;
+    }
+    return true;
+}
+__device__ __forceinline__ bool mbar_wait_sleep(uint64_t* bar, uint32_t parity, long long limit)
+{
+    if (mbar_try_wait_sleep(bar, parity)) return true;
+    const long long t0 = clock64();
+    while (!mbar_try_wait_sleep(bar, parity)) {
         if (clock64() - t0 > limit) return false;
     }
     return true;
