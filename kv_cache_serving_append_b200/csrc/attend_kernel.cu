@@ -10,26 +10,26 @@
 // definition, stated in rtv.h.
 //
 // One CTA = two 128-row query tiles of one head, sharing every K/V tile it
-// loads; 12 warps:
+// loads; KV tiles of 64 keys; 12 warps:
 //   warp 0     TMA producer: both Q tiles once; per KV tile the K and V code
 //              tiles at (ring slot * H + head, token tile) and their scales.
-//   warps 1,3  MMA issuers, one per query tile t (warp 1 also owns TMEM).  Per
-//              KV tile j: S_t = Q_t K_j^T (kind::f8f6f4, E4M3 x E4M3 -> f32 in
-//              TMEM), then O_t += P_t V16_j (kind::f16, P_t read from TMEM where
-//              it overwrote S_t, V16 from shared memory).  Two independent
-//              issuers let one tile's softmax run while the other tile's MMAs
-//              are on the tensor core, with blocking waits and no polling.
+//   warps 1,3  MMA issuers, one per query tile t (warp 1 also owns TMEM).
+//              S_t,b = Q_t K_j^T (kind::f8f6f4, E4M3 x E4M3 -> f32 in TMEM,
+//              b = j mod 2: two S buffers per query tile), O_t += P_t,b V16_j
+//              (kind::f16, P read from TMEM where it overwrote S_t,b, V16
+//              from shared memory).  With two S buffers the softmax of KV tile
+//              j+1 runs while PV(j) and QK(j+2) execute.
 //   warp 2     widens the V code tile to f16 (exact) in the MN-major layout
 //              the PV MMA reads.
 //   warps 4-7  softmax of query tile 0, warps 8-11 of query tile 1; one query
-//              row per thread, the tile's 128 scores held in registers (one
-//              TMEM round trip per KV tile): s*scale_k, running max, exp2, row sum,
-//              P = p*scale_v/Sv in f16 written back over S; lazy O rescaling
-//              only when the running max grows by more than 2^8.
-// TMEM columns: S_0 [0,128), S_1 [128,256), O_0 [256,256+D), O_1 [384,384+D).
-// QK_t(j+1) is issued only once PV_t(j) has completed (its mbarrier), so the
-// P that PV_t(j) reads is never overwritten early and O_t is idle whenever
-// the softmax of tile t runs (the rescale needs no wait).
+//              row per thread, the tile's 64 scores in registers: s*scale_k,
+//              running max, exp2, row sum, P = p*scale_v/Sv in f16 written
+//              back over S; lazy O rescaling only when the running max grows
+//              by more than 2^8.  The two warpgroups take turns on their exp
+//              phases, so each runs with the exp unit (16/clk/SM) to itself.
+// TMEM columns: S_t,b at 64*(2t+b) (64 columns each), O_0 [256,256+D),
+// O_1 [384,384+D).  QK(j+2) overwrites S_t,b only after PV(j), which reads
+// P_t,b out of it, has completed.
 //
 // Logical-to-physical frame order is resolved in the TMA coordinates: the
 // kernel receives the key set as a list of ring slots -- no gather, no copy.
@@ -58,32 +58,34 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kBM = 128;        // query rows per query tile
-constexpr int kQT = 2;          // query tiles per CTA
-constexpr int kBN = 128;        // keys per KV tile
-constexpr int kStages = 3;      // K/V code tile stages
+constexpr int kBM = kAttendRows;   // query rows per query tile
+constexpr int kQT = 2;             // query tiles per CTA
+constexpr int kBN = kAttendKeys;   // keys per KV tile
+constexpr int kStages = 6;         // K/V code tile stages
+constexpr int kNV16 = 4;           // f16 V tile buffers
 constexpr int kThreads = 384;
 constexpr uint32_t kTmemCols = 512;
 constexpr float kLazyRescaleLog2 = 8.0f;   // rescale O only when the max grows by > 2^8
 
-__host__ __device__ constexpr uint32_t col_s(int t) { return 128u * t; }
+__host__ __device__ constexpr uint32_t col_s(int t, int b) { return 64u * (2 * t + b); }
 __host__ __device__ constexpr uint32_t col_o(int t) { return 256u + 128u * t; }
 
 template <int D>
 struct Smem {
-    static constexpr int kTileBytes = kBM * D;            // one FP8 code tile (Q, K or V)
+    static constexpr int kQBytes = kBM * D;               // one FP8 query tile
+    static constexpr int kKVBytes = kBN * D;              // one FP8 K or V tile
     static constexpr int kV16Bytes = kBN * D * 2;          // one f16 V tile
-    alignas(1024) uint8_t q[kQT][kTileBytes];
-    alignas(1024) uint8_t k[kStages][kTileBytes];
-    alignas(1024) uint8_t v8[kStages][kTileBytes];
-    alignas(1024) uint8_t v16[2][kV16Bytes];
+    alignas(1024) uint8_t q[kQT][kQBytes];
+    alignas(1024) uint8_t k[kStages][kKVBytes];
+    alignas(1024) uint8_t v8[kStages][kKVBytes];
+    alignas(1024) uint8_t v16[kNV16][kV16Bytes];
     alignas(128) float sk[kStages][kBN];
     alignas(128) float sv[kStages][kBN];
     uint64_t q_full;
     uint64_t k_full[kStages];
     uint64_t kv_empty[kStages];
-    uint64_t s_full[kQT], p_ready[kQT], pv_done[kQT];
-    uint64_t v16_ready[2], tile_done[2];
+    uint64_t s_full[kQT][2], p_ready[kQT][2], pv_done[kQT][2];
+    uint64_t v16_ready[kNV16], tile_done[kNV16];
     uint64_t drain[kQT];
     uint64_t exp_turn[kQT];   // alternation of the two softmax warpgroups' exp phases
     uint32_t tmem_base;
@@ -151,7 +153,7 @@ __device__ __forceinline__ bool warp_wait_sleep(uint64_t* bar, uint32_t parity, 
     return __all_sync(0xffffffffu, mbar_wait_sleep(bar, parity, limit));
 }
 
-// Pass 1 of a KV tile, on the 128 scores of this thread's row held in
+// Pass 1 of a KV tile, on the kBN scores of this thread's row held in
 // registers: u = s * scale_k (written back over s, in pairs) and the row max of
 // u over the valid keys.  kMask: tile with fewer than 128 valid keys.
 template <bool kMask>
@@ -161,8 +163,7 @@ __device__ __forceinline__ float tile_row_max(uint32_t* sr, const float* sk, int
     float mt0 = -INFINITY, mt1 = -INFINITY;
 #pragma unroll
     for (int k4 = 0; k4 < kBN / 4; ++k4) {
-        // keep the scale loads to one 32-key chunk in flight (registers: the
-        // 128 scores already occupy most of the thread's budget)
+        // keep the scale loads to one 32-key chunk in flight (register budget)
         if ((k4 & 7) == 0) asm volatile("" ::: "memory");
         const float4 kk = sk4[k4];
         const uint64_t u0 = mul2(pack2(__uint_as_float(sr[4 * k4]), __uint_as_float(sr[4 * k4 + 1])),
@@ -263,13 +264,15 @@ attend_kernel(const __grid_constant__ AttendParams p, const __grid_constant__ CU
             mbar_init(&sm.kv_empty[s], n_qt);
         }
         for (int t = 0; t < kQT; ++t) {
-            mbar_init(&sm.s_full[t], 1);
-            mbar_init(&sm.p_ready[t], 128);
-            mbar_init(&sm.pv_done[t], 1);
+            for (int b = 0; b < 2; ++b) {
+                mbar_init(&sm.s_full[t][b], 1);
+                mbar_init(&sm.p_ready[t][b], 128);
+                mbar_init(&sm.pv_done[t][b], 1);
+            }
             mbar_init(&sm.drain[t], 1);
             mbar_init(&sm.exp_turn[t], 128);
         }
-        for (int b = 0; b < 2; ++b) {
+        for (int b = 0; b < kNV16; ++b) {
             mbar_init(&sm.v16_ready[b], 32);
             mbar_init(&sm.tile_done[b], n_qt);
         }
@@ -300,8 +303,8 @@ attend_kernel(const __grid_constant__ AttendParams p, const __grid_constant__ CU
         if (warp == 0) {
             // ------------------------------------------------------ producer --
             if (lane == 0 && !p.debug_wait_fault) {
-                constexpr uint32_t kTileBytes = Smem<D>::kTileBytes;
-                mbar_arrive_expect_tx(&sm.q_full, kQT * kTileBytes);
+                constexpr uint32_t kQBytes = Smem<D>::kQBytes, kKVBytes = Smem<D>::kKVBytes;
+                mbar_arrive_expect_tx(&sm.q_full, kQT * kQBytes);
                 for (int t = 0; t < kQT; ++t) tma_load_3d(sm.q[t], &map_q, &sm.q_full, 0, q0 + t * kBM, h);
                 int issued = 0;
                 for (int j = 0; j < n_tiles; ++j) {
@@ -314,7 +317,7 @@ attend_kernel(const __grid_constant__ AttendParams p, const __grid_constant__ CU
                     const int fi = j / p.tiles_per_frame;
                     const int t0 = (j - fi * p.tiles_per_frame) * kBN;
                     const int row = p.slot[fi] * H + h;
-                    mbar_arrive_expect_tx(&sm.k_full[st], 2 * kTileBytes + 2 * kBN * 4);
+                    mbar_arrive_expect_tx(&sm.k_full[st], 2 * kKVBytes + 2 * kBN * 4);
                     tma_load_3d(sm.k[st], &map_k, &sm.k_full[st], 0, t0, row);
                     tma_load_3d(sm.v8[st], &map_v, &sm.k_full[st], 0, t0, row);
                     tma_load_2d(sm.sk[st], &map_sk, &sm.k_full[st], t0, row);
@@ -337,32 +340,41 @@ attend_kernel(const __grid_constant__ AttendParams p, const __grid_constant__ CU
                 constexpr uint32_t kSw = D == 128 ? kSwizzle128 : kSwizzle64;
                 constexpr uint32_t kSbo = D == 128 ? 1024 : 512;
                 const uint32_t q_addr = smem_u32(sm.q[t]);
-                if (!mbar_wait(&sm.q_full, 0, limit)) fail = true;
-                for (int j = 0; j < n_tiles && !fail; ++j) {
-                    // S_t = Q_t K_j^T once K_j has landed and PV_t(j-1) (which reads
-                    // P_t out of the S_t columns) has completed
-                    if (!mbar_wait(&sm.k_full[j % kStages], (j / kStages) & 1, limit)) { fail = true; break; }
-                    if (j > 0 && !mbar_wait(&sm.pv_done[t], (j - 1) & 1, limit)) { fail = true; break; }
+                // S_t,b = Q_t K_j^T, b = j & 1, once K_j has landed
+                auto issue_qk = [&](int j) -> bool {
+                    if (!mbar_wait(&sm.k_full[j % kStages], (j / kStages) & 1, limit)) return false;
                     tc_fence_after();
                     const uint32_t k_addr = smem_u32(sm.k[j % kStages]);
-    #pragma unroll
+#pragma unroll
                     for (int kk = 0; kk < D / 32; ++kk)
-                        mma_f8_ss(tmem + col_s(t), smem_desc(q_addr + kk * 32, 16, kSbo, kSw),
+                        mma_f8_ss(tmem + col_s(t, j & 1), smem_desc(q_addr + kk * 32, 16, kSbo, kSw),
                                   smem_desc(k_addr + kk * 32, 16, kSbo, kSw), kQK, kk > 0);
-                    tc_commit(&sm.s_full[t]);
-                    // O_t += P_t V_j once the softmax wrote P_t and V_j is widened
-                    if (!mbar_wait(&sm.p_ready[t], j & 1, limit)) { fail = true; break; }
-                    if (!mbar_wait(&sm.v16_ready[j & 1], (j >> 1) & 1, limit)) { fail = true; break; }
+                    tc_commit(&sm.s_full[t][j & 1]);
+                    return true;
+                };
+                if (!mbar_wait(&sm.q_full, 0, limit)) fail = true;
+                if (!fail && !issue_qk(0)) fail = true;
+                if (!fail && n_tiles > 1 && !issue_qk(1)) fail = true;
+                for (int j = 0; j < n_tiles && !fail; ++j) {
+                    const int b = j & 1, vb = j % kNV16;
+                    // O_t += P_t,b V_j once the softmax wrote P and V_j is widened
+                    if (!mbar_wait(&sm.p_ready[t][b], (j >> 1) & 1, limit)) { fail = true; break; }
+                    if (!mbar_wait(&sm.v16_ready[vb], (j / kNV16) & 1, limit)) { fail = true; break; }
                     tc_fence_after();
-                    const uint32_t v_addr = smem_u32(sm.v16[j & 1]);
-    #pragma unroll
+                    const uint32_t v_addr = smem_u32(sm.v16[vb]);
+#pragma unroll
                     for (int kk = 0; kk < kBN / 16; ++kk)
-                        mma_f16_ts(tmem + col_o(t), tmem + col_s(t) + kk * 8,
-                                   smem_desc(v_addr + kk * 2048, 16384, 1024, kSwizzle128), kPV,
+                        mma_f16_ts(tmem + col_o(t), tmem + col_s(t, b) + kk * 8,
+                                   smem_desc(v_addr + kk * 2048, kBN * 128, 1024, kSwizzle128), kPV,
                                    (j > 0 || kk > 0) ? 1u : 0u);
-                    tc_commit(&sm.pv_done[t]);
+                    tc_commit(&sm.pv_done[t][b]);
                     tc_commit(&sm.kv_empty[j % kStages]);
-                    tc_commit(&sm.tile_done[j & 1]);
+                    tc_commit(&sm.tile_done[vb]);
+                    // S_t,b is free again once PV(j) has read P out of it
+                    if (j + 2 < n_tiles) {
+                        if (!mbar_wait(&sm.pv_done[t][b], (j >> 1) & 1, limit)) { fail = true; break; }
+                        if (!issue_qk(j + 2)) { fail = true; break; }
+                    }
                 }
                 // drain: all MMAs issued by this thread complete before TMEM is freed
                 tc_commit(&sm.drain[t]);
@@ -377,9 +389,10 @@ attend_kernel(const __grid_constant__ AttendParams p, const __grid_constant__ CU
             constexpr int kNB = D / 64;                 // 64-element blocks per key row
             const int rl = lane & 7, cq = lane >> 3;
             for (int j = 0; j < n_tiles; ++j) {
-                const int st = j % kStages, b = j & 1;
+                const int st = j % kStages, b = j % kNV16;
                 if (!warp_wait_sleep(&sm.k_full[st], (j / kStages) & 1, limit)) { fail = true; break; }
-                if (j >= 2 && !warp_wait_sleep(&sm.tile_done[b], ((j >> 1) - 1) & 1, limit)) { fail = true; break; }
+                if (j >= kNV16 &&
+                    !warp_wait_sleep(&sm.tile_done[b], ((j / kNV16) - 1) & 1, limit)) { fail = true; break; }
                 const uint8_t* src = sm.v8[st];
                 uint8_t* dst = sm.v16[b];
     #pragma unroll 4
@@ -412,7 +425,6 @@ attend_kernel(const __grid_constant__ AttendParams p, const __grid_constant__ CU
         if (t < n_qt) {
             const int row = (warp & 3) * 32 + lane;     // TMEM lane == query row in tile
             const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
-            const uint32_t t_s = tmem + lane_off + col_s(t);
             const uint32_t t_o = tmem + lane_off + col_o(t);
             const int qrow = q0 + t * kBM + row;
             const bool row_ok = qrow < p.M;
@@ -437,11 +449,12 @@ attend_kernel(const __grid_constant__ AttendParams p, const __grid_constant__ CU
             float l = 0.f;         // running sum of p / Sv
             const uint64_t c2c2 = pack2(c2, c2);
             for (int j = 0; j < n_tiles && !fail; ++j) {
-                const int st = j % kStages;
+                const int st = j % kStages, b = j & 1;
                 const int fi = j / p.tiles_per_frame;
                 const int nv = min(kBN, p.T - (j - fi * p.tiles_per_frame) * kBN);
+                const uint32_t t_s = tmem + lane_off + col_s(t, b);
                 if (!warp_wait(&sm.k_full[st], (j / kStages) & 1, limit)) { fail = true; break; }
-                if (!warp_wait(&sm.s_full[t], j & 1, limit)) { fail = true; break; }
+                if (!warp_wait(&sm.s_full[t][b], (j >> 1) & 1, limit)) { fail = true; break; }
                 tc_fence_after();
                 uint32_t sr[kBN];
 #pragma unroll
@@ -454,13 +467,15 @@ attend_kernel(const __grid_constant__ AttendParams p, const __grid_constant__ CU
                 if (j == 0) {
                     m = m_new;   // first tile: O not yet written
                 } else if (__any_sync(0xffffffffu, (m_new - m) * c2 > kLazyRescaleLog2)) {
-                    // Warp-uniform decision (the TMEM load/store below are
-                    // warp-collective); every lane moves to its own new max
-                    // (alpha = 1 where it did not grow).  PV_t(j-1) completed
-                    // before S_t(j) was computed, so O_t is not being written.
+                    // Warp-uniform decision (the wait and the TMEM load/store
+                    // below are warp-collective); every lane moves to its own
+                    // new max (alpha = 1 where it did not grow).  O_t holds PV
+                    // up to tile j-1: wait for it to complete, scale in place.
                     const float alpha = ex2((m - m_new) * c2);
                     l *= alpha;
                     m = m_new;
+                    if (!warp_wait(&sm.pv_done[t][(j - 1) & 1], ((j - 1) >> 1) & 1, limit)) { fail = true; break; }
+                    tc_fence_after();
 #pragma unroll 1
                     for (int c = 0; c < D / 32; ++c) {
                         uint32_t o[32];
@@ -486,9 +501,10 @@ attend_kernel(const __grid_constant__ AttendParams p, const __grid_constant__ CU
                 if (pingpong) mbar_arrive(&sm.exp_turn[1 - t]);
                 tc_wait_st();
                 tc_fence_before();
-                mbar_arrive(&sm.p_ready[t]);
+                mbar_arrive(&sm.p_ready[t][b]);
             }
-            if (!fail && !warp_wait(&sm.pv_done[t], (n_tiles - 1) & 1, limit)) fail = true;
+            if (!fail && !warp_wait(&sm.pv_done[t][(n_tiles - 1) & 1], ((n_tiles - 1) >> 1) & 1, limit))
+                fail = true;
             if (!fail) {
                 tc_fence_after();
                 const float norm = 1.f / l;

@@ -167,14 +167,14 @@ bool build_maps(rtv_cache* c)
         {   // Q codes [H][q_rows][D]
             cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)q_rows, (cuuint64_t)H};
             cuuint64_t st[2] = {(cuuint64_t)D, (cuuint64_t)q_rows * D};
-            cuuint32_t box[3] = {(cuuint32_t)D, 128, 1};
+            cuuint32_t box[3] = {(cuuint32_t)D, (cuuint32_t)kAttendRows, 1};
             if (!encode(&m[0], CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, c->buf + L.q_codes, dims, st, box, sw))
                 return false;
         }
         for (int kv = 0; kv < 2; ++kv) {   // K/V codes [S*H][T][D]
             cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)T, (cuuint64_t)S * H};
             cuuint64_t st[2] = {(cuuint64_t)D, (cuuint64_t)T * D};
-            cuuint32_t box[3] = {(cuuint32_t)D, 128, 1};
+            cuuint32_t box[3] = {(cuuint32_t)D, (cuuint32_t)kAttendKeys, 1};
             if (!encode(&m[1 + kv], CU_TENSOR_MAP_DATA_TYPE_UINT8, 3,
                         c->buf + (kv ? L.v_codes : L.k_codes), dims, st, box, sw))
                 return false;
@@ -182,7 +182,7 @@ bool build_maps(rtv_cache* c)
         for (int kv = 0; kv < 2; ++kv) {   // scales [S*H][scale_pitch] (first T used)
             cuuint64_t dims[2] = {(cuuint64_t)T, (cuuint64_t)S * H};
             cuuint64_t st[1] = {(cuuint64_t)L.scale_pitch * 4};
-            cuuint32_t box[2] = {128, 1};
+            cuuint32_t box[2] = {(cuuint32_t)kAttendKeys, 1};
             if (!encode(&m[3 + kv], CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2,
                         c->buf + (kv ? L.v_scales : L.k_scales), dims, st, box,
                         CU_TENSOR_MAP_SWIZZLE_NONE))
@@ -398,7 +398,7 @@ rtv_status rtv_attend(rtv_cache* c, int layer, void* out, int out_dtype, void* s
     p.H = c->H; p.D = c->D; p.T = c->T; p.M = n * c->T;
     p.q_scale_pitch = L.q_scale_pitch;
     p.out_bf16 = out_dtype == RTV_OUT_BF16;
-    p.tiles_per_frame = (c->T + 127) / 128;
+    p.tiles_per_frame = (c->T + kAttendKeys - 1) / kAttendKeys;
     int nk = 0;
     for (int s : c->visible_slots) p.slot[nk++] = s;
     for (int f = 0; f < n; ++f) p.slot[nk++] = staged_slot(c, f);

@@ -15,6 +15,11 @@ constexpr int kMaxSlots = RTV_MAX_SLOTS;
 constexpr int kMaxHeads = 256;     // append kernel keeps one V-scale max per head in smem
 constexpr int kMaxRopeHalf = 32;   // rope_t / 2 <= 32 (frame-axis table travels in params)
 
+// Attention tiling shared by the kernel and the host-side TMA descriptors:
+// 128 query rows per query tile, 64 keys per KV tile.
+constexpr int kAttendRows = 128;
+constexpr int kAttendKeys = 64;
+
 // Device error word bits.
 constexpr uint32_t kErrTimeout = 1u;
 
@@ -49,7 +54,7 @@ struct AttendParams {
     int q_scale_pitch;
     int out_bf16;
     int n_frames_keys;             // frames in the key set
-    int tiles_per_frame;           // ceil(T / 128)
+    int tiles_per_frame;           // ceil(T / kAttendKeys)
     int debug_wait_fault;          // 1: producer never arms the first barrier
     long long wait_limit;          // per-wait limit in clock cycles
     int slot[kMaxSlots];           // key set, logical order
