@@ -66,6 +66,7 @@ constexpr int kNV16 = 4;           // f16 V tile buffers
 constexpr int kThreads = 384;
 constexpr uint32_t kTmemCols = 512;
 constexpr float kLazyRescaleLog2 = 8.0f;   // rescale O only when the max grows by > 2^8
+constexpr uint32_t kBarTurn0 = 1, kBarTurn1 = 2;   // named barriers: warpgroup 0 / 1 may start its exp phase
 
 __host__ __device__ constexpr uint32_t col_s(int t, int b) { return 64u * (2 * t + b); }
 __host__ __device__ constexpr uint32_t col_o(int t) { return 256u + 128u * t; }
@@ -87,7 +88,6 @@ struct Smem {
     uint64_t s_full[kQT][2], p_ready[kQT][2], pv_done[kQT][2];
     uint64_t v16_ready[kNV16], tile_done[kNV16];
     uint64_t drain[kQT];
-    uint64_t exp_turn[kQT];   // alternation of the two softmax warpgroups' exp phases
     uint32_t tmem_base;
 };
 
@@ -270,7 +270,6 @@ attend_kernel(const __grid_constant__ AttendParams p, const __grid_constant__ CU
                 mbar_init(&sm.pv_done[t][b], 1);
             }
             mbar_init(&sm.drain[t], 1);
-            mbar_init(&sm.exp_turn[t], 128);
         }
         for (int b = 0; b < kNV16; ++b) {
             mbar_init(&sm.v16_ready[b], 32);
@@ -342,7 +341,7 @@ attend_kernel(const __grid_constant__ AttendParams p, const __grid_constant__ CU
                 const uint32_t q_addr = smem_u32(sm.q[t]);
                 // S_t,b = Q_t K_j^T, b = j & 1, once K_j has landed
                 auto issue_qk = [&](int j) -> bool {
-                    if (!mbar_wait(&sm.k_full[j % kStages], (j / kStages) & 1, limit)) return false;
+                    if (!mbar_wait_backoff(&sm.k_full[j % kStages], (j / kStages) & 1, limit)) return false;
                     tc_fence_after();
                     const uint32_t k_addr = smem_u32(sm.k[j % kStages]);
 #pragma unroll
@@ -352,14 +351,14 @@ attend_kernel(const __grid_constant__ AttendParams p, const __grid_constant__ CU
                     tc_commit(&sm.s_full[t][j & 1]);
                     return true;
                 };
-                if (!mbar_wait(&sm.q_full, 0, limit)) fail = true;
+                if (!mbar_wait_backoff(&sm.q_full, 0, limit)) fail = true;
                 if (!fail && !issue_qk(0)) fail = true;
                 if (!fail && n_tiles > 1 && !issue_qk(1)) fail = true;
                 for (int j = 0; j < n_tiles && !fail; ++j) {
                     const int b = j & 1, vb = j % kNV16;
                     // O_t += P_t,b V_j once the softmax wrote P and V_j is widened
-                    if (!mbar_wait(&sm.p_ready[t][b], (j >> 1) & 1, limit)) { fail = true; break; }
-                    if (!mbar_wait(&sm.v16_ready[vb], (j / kNV16) & 1, limit)) { fail = true; break; }
+                    if (!mbar_wait_backoff(&sm.p_ready[t][b], (j >> 1) & 1, limit)) { fail = true; break; }
+                    if (!mbar_wait_backoff(&sm.v16_ready[vb], (j / kNV16) & 1, limit)) { fail = true; break; }
                     tc_fence_after();
                     const uint32_t v_addr = smem_u32(sm.v16[vb]);
 #pragma unroll
@@ -372,13 +371,13 @@ attend_kernel(const __grid_constant__ AttendParams p, const __grid_constant__ CU
                     tc_commit(&sm.tile_done[vb]);
                     // S_t,b is free again once PV(j) has read P out of it
                     if (j + 2 < n_tiles) {
-                        if (!mbar_wait(&sm.pv_done[t][b], (j >> 1) & 1, limit)) { fail = true; break; }
+                        if (!mbar_wait_backoff(&sm.pv_done[t][b], (j >> 1) & 1, limit)) { fail = true; break; }
                         if (!issue_qk(j + 2)) { fail = true; break; }
                     }
                 }
                 // drain: all MMAs issued by this thread complete before TMEM is freed
                 tc_commit(&sm.drain[t]);
-                if (!mbar_wait(&sm.drain[t], 0, limit)) fail = true;
+                if (!mbar_wait_backoff(&sm.drain[t], 0, limit)) fail = true;
             }
         } else if (warp == 2) {
             // ------------------------------------------- V widening (FP8->f16) --
@@ -448,6 +447,8 @@ attend_kernel(const __grid_constant__ AttendParams p, const __grid_constant__ CU
             float m = -INFINITY;   // running max of s * scale_k (lazy)
             float l = 0.f;         // running sum of p / Sv
             const uint64_t c2c2 = pack2(c2, c2);
+            const bool pingpong = n_qt == 2;
+            int arrived = 0;       // KV tiles whose turn-barrier arrival this warpgroup has made
             for (int j = 0; j < n_tiles && !fail; ++j) {
                 const int st = j % kStages, b = j & 1;
                 const int fi = j / p.tiles_per_frame;
@@ -487,22 +488,32 @@ attend_kernel(const __grid_constant__ AttendParams p, const __grid_constant__ CU
                     }
                 }
                 // pass 2: p / Sv = 2^(u*c2 - m*c2 - log2 Sv); P = (p / Sv) * scale_v.
-                // With two query tiles the warpgroups take turns (tile 0 of
-                // KV tile j, tile 1 of j, tile 0 of j+1, ...): each exp phase
-                // then runs with the exp unit to itself, and one tile's PV and
-                // next QK overlap the other tile's exp phase.
-                const bool pingpong = n_qt == 2;
-                if (pingpong && (t == 1 || j > 0) &&
-                    !warp_wait(&sm.exp_turn[t], (t == 1 ? j : j - 1) & 1, limit)) { fail = true; break; }
+                // With two query tiles the warpgroups take turns (tile 0 of KV
+                // tile j, tile 1 of j, tile 0 of j+1, ...) through two named
+                // barriers: each exp phase runs with the exp unit to itself,
+                // and the waiting warpgroup is blocked in hardware, taking no
+                // issue slots from the one computing.
+                if (pingpong && (t == 1 || j > 0)) named_bar_sync(t == 0 ? kBarTurn0 : kBarTurn1, 256);
                 const float neg = -(m * c2 + log2_sv);
                 const uint64_t neg2 = pack2(neg, neg);
                 l += nv == kBN ? tile_make_p<false>(sr, t_s, sm.sv[st], c2c2, neg2, nv)
                                : tile_make_p<true>(sr, t_s, sm.sv[st], c2c2, neg2, nv);
-                if (pingpong) mbar_arrive(&sm.exp_turn[1 - t]);
+                if (pingpong && (t == 0 || j + 1 < n_tiles)) named_bar_arrive(t == 0 ? kBarTurn1 : kBarTurn0, 256);
+                arrived = j + 1;
                 tc_wait_st();
                 tc_fence_before();
                 mbar_arrive(&sm.p_ready[t][b]);
             }
+            // On failure (which can only happen before a tile's turn sync),
+            // still contribute to every remaining generation of both turn
+            // barriers -- an arrive in place of each sync, then the tile's own
+            // arrive -- so every barrier generation completes exactly as in a
+            // normal run and no warp can block in a named-barrier sync.
+            if (pingpong)
+                for (int j = arrived; j < n_tiles; ++j) {
+                    if (t == 1 || j > 0) named_bar_arrive(t == 0 ? kBarTurn0 : kBarTurn1, 256);
+                    if (t == 0 || j + 1 < n_tiles) named_bar_arrive(t == 0 ? kBarTurn1 : kBarTurn0, 256);
+                }
             if (!fail && !warp_wait(&sm.pv_done[t][(n_tiles - 1) & 1], ((n_tiles - 1) >> 1) & 1, limit))
                 fail = true;
             if (!fail) {

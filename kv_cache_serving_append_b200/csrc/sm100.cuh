@@ -89,6 +89,18 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, long l
     }
     return true;
 }
+// Spin with a short back-off: a few instructions per ~64 ns instead of a tight
+// loop (for single-thread roles whose wake-up latency has slack).
+__device__ __forceinline__ bool mbar_wait_backoff(uint64_t* bar, uint32_t parity, long long limit)
+{
+    if (mbar_try_wait(bar, parity)) return true;
+    const long long t0 = clock64();
+    while (!mbar_try_wait(bar, parity)) {
+        __nanosleep(64);
+        if (clock64() - t0 > limit) return false;
+    }
+    return true;
+}
 __device__ __forceinline__ bool mbar_wait_sleep(uint64_t* bar, uint32_t parity, long long limit)
 {
     if (mbar_try_wait_sleep(bar, parity)) return true;
@@ -97,6 +109,17 @@ __device__ __forceinline__ bool mbar_wait_sleep(uint64_t* bar, uint32_t parity, 
         if (clock64() - t0 > limit) return false;
     }
     return true;
+}
+
+// Named barriers (hardware-blocking, no polling).  Used only where every
+// participant's arrivals are guaranteed, on the failure path too.
+__device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t nthreads)
+{
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+__device__ __forceinline__ void named_bar_arrive(uint32_t id, uint32_t nthreads)
+{
+    asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
 // ------------------------------------------------------------------ TMA --
