@@ -65,7 +65,8 @@ constexpr int kStages = 6;         // K/V code tile stages
 constexpr int kNV16 = 4;           // f16 V tile buffers
 constexpr int kThreads = 384;
 constexpr uint32_t kTmemCols = 512;
-constexpr float kLazyRescaleLog2 = 8.0f;   // rescale O only when the max grows by > 2^8
+constexpr float kLazyRescaleLog2 = 8.0f;   // move the running max when a tile's p grows past 2^8
+constexpr float kRedoLog2 = 15.0f;         // redo a tile whose p would exceed 2^15 (f16 P range)
 constexpr uint32_t kBarTurn0 = 1, kBarTurn1 = 2;   // named barriers: warpgroup 0 / 1 may start its exp phase
 
 __host__ __device__ constexpr uint32_t col_s(int t, int b) { return 64u * (2 * t + b); }
@@ -153,72 +154,76 @@ __device__ __forceinline__ bool warp_wait_sleep(uint64_t* bar, uint32_t parity, 
     return __all_sync(0xffffffffu, mbar_wait_sleep(bar, parity, limit));
 }
 
-// Pass 1 of a KV tile, on the kBN scores of this thread's row held in
-// registers: u = s * scale_k (written back over s, in pairs) and the row max of
-// u over the valid keys.  kMask: tile with fewer than 128 valid keys.
+// Row max of u = s * scale_k over the valid keys of a KV tile (the kBN scores
+// of this thread's row are in registers).  Used for the first KV tile and
+// when a tile's scores outgrow the running max by more than f16 P allows.
 template <bool kMask>
-__device__ __forceinline__ float tile_row_max(uint32_t* sr, const float* sk, int nv)
+__device__ __forceinline__ float tile_row_max(const uint32_t* sr, const float* sk, int nv)
 {
     const float4* sk4 = reinterpret_cast<const float4*>(sk);
-    float mt0 = -INFINITY, mt1 = -INFINITY;
+    float mt[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
     for (int k4 = 0; k4 < kBN / 4; ++k4) {
-        // keep the scale loads to one 32-key chunk in flight (register budget)
-        if ((k4 & 7) == 0) asm volatile("" ::: "memory");
         const float4 kk = sk4[k4];
-        const uint64_t u0 = mul2(pack2(__uint_as_float(sr[4 * k4]), __uint_as_float(sr[4 * k4 + 1])),
-                                 pack2(kk.x, kk.y));
-        const uint64_t u1 = mul2(pack2(__uint_as_float(sr[4 * k4 + 2]), __uint_as_float(sr[4 * k4 + 3])),
-                                 pack2(kk.z, kk.w));
         float a, b, c, d;
-        unpack2(u0, a, b);
-        unpack2(u1, c, d);
-        sr[4 * k4] = __float_as_uint(a);
-        sr[4 * k4 + 1] = __float_as_uint(b);
-        sr[4 * k4 + 2] = __float_as_uint(c);
-        sr[4 * k4 + 3] = __float_as_uint(d);
+        unpack2(mul2(pack2(__uint_as_float(sr[4 * k4]), __uint_as_float(sr[4 * k4 + 1])),
+                     pack2(kk.x, kk.y)), a, b);
+        unpack2(mul2(pack2(__uint_as_float(sr[4 * k4 + 2]), __uint_as_float(sr[4 * k4 + 3])),
+                     pack2(kk.z, kk.w)), c, d);
+        float& m0 = mt[(k4 & 1) * 2];
+        float& m1 = mt[(k4 & 1) * 2 + 1];
         if (!kMask) {
-            mt0 = max3(mt0, a, b);
-            mt1 = max3(mt1, c, d);
+            m0 = max3(m0, a, b);
+            m1 = max3(m1, c, d);
         } else {
             const int k = 4 * k4;
-            if (k < nv) mt0 = fmaxf(mt0, a);
-            if (k + 1 < nv) mt1 = fmaxf(mt1, b);
-            if (k + 2 < nv) mt0 = fmaxf(mt0, c);
-            if (k + 3 < nv) mt1 = fmaxf(mt1, d);
+            if (k < nv) m0 = fmaxf(m0, a);
+            if (k + 1 < nv) m1 = fmaxf(m1, b);
+            if (k + 2 < nv) m0 = fmaxf(m0, c);
+            if (k + 3 < nv) m1 = fmaxf(m1, d);
         }
     }
-    return fmaxf(mt0, mt1);
+    return fmaxf(fmaxf(mt[0], mt[1]), fmaxf(mt[2], mt[3]));
 }
 
-// Pass 2 of a KV tile: p/Sv = 2^(u*c2 + neg), P = (p/Sv) * scale_v packed to
-// f16 pairs and written over S in TMEM (keys [32c, 32c+32) -> P columns
-// [16c, 16c+16); all of S was read before).  Returns the row sum of p/Sv.
+// One pass over a KV tile (the kBN scores of this thread's row in registers):
+// u = s * scale_k, x = u*c2 + neg (= (u - m)*c2 - log2 Sv for the running max
+// m), p/Sv = 2^x, P = (p/Sv) * scale_v packed to f16 pairs and written over S
+// in TMEM (keys [32c, 32c+32) -> P columns [16c, 16c+16); S is already in
+// registers).  Returns the row sum of p/Sv; xmax = max of x over valid keys,
+// from which the caller sees whether the tile outgrew the running max.
 template <bool kMask>
-__device__ __forceinline__ float tile_make_p(const uint32_t* sr, uint32_t t_s, const float* sv,
-                                             uint64_t c2c2, uint64_t neg2, int nv)
+__device__ __forceinline__ float tile_exp(const uint32_t* sr, uint32_t t_s, const float* sk,
+                                          const float* sv, uint64_t c2c2, uint64_t neg2, int nv,
+                                          float& xmax)
 {
+    const float4* sk4 = reinterpret_cast<const float4*>(sk);
     const float4* sv4 = reinterpret_cast<const float4*>(sv);
-    uint64_t ls2 = pack2(0.f, 0.f);
+    // independent partial row sums and maxima: short dependency chains
+    uint64_t ls2[4] = {pack2(0.f, 0.f), pack2(0.f, 0.f), pack2(0.f, 0.f), pack2(0.f, 0.f)};
+    float xm[2] = {-INFINITY, -INFINITY};
 #pragma unroll
     for (int c = 0; c < kBN / 32; ++c) {
         uint32_t pk[16];
 #pragma unroll
         for (int k4 = 0; k4 < 8; ++k4) {
+            const float4 kk = sk4[c * 8 + k4];
             const float4 vv = sv4[c * 8 + k4];
 #pragma unroll
             for (int hh = 0; hh < 2; ++hh) {
                 const int k = c * 32 + 4 * k4 + 2 * hh;
+                const uint64_t u = mul2(pack2(__uint_as_float(sr[k]), __uint_as_float(sr[k + 1])),
+                                        hh ? pack2(kk.z, kk.w) : pack2(kk.x, kk.y));
                 float x0, x1;
-                unpack2(fma2(pack2(__uint_as_float(sr[k]), __uint_as_float(sr[k + 1])), c2c2, neg2),
-                        x0, x1);
-                float p0 = ex2(x0), p1 = ex2(x1);
+                unpack2(fma2(u, c2c2, neg2), x0, x1);
                 if (kMask) {
-                    if (k >= nv) p0 = 0.f;
-                    if (k + 1 >= nv) p1 = 0.f;
+                    if (k >= nv) x0 = -INFINITY;
+                    if (k + 1 >= nv) x1 = -INFINITY;
                 }
+                xm[hh] = max3(xm[hh], x0, x1);
+                const float p0 = ex2(x0), p1 = ex2(x1);   // ex2(-inf) = 0 for masked keys
                 const uint64_t pp = pack2(p0, p1);
-                ls2 = add2(ls2, pp);
+                ls2[(k >> 1) & 3] = add2(ls2[(k >> 1) & 3], pp);
                 float q0, q1;
                 unpack2(mul2(pp, hh ? pack2(vv.z, vv.w) : pack2(vv.x, vv.y)), q0, q1);
                 __half2 hv = __floats2half2_rn(q0, q1);
@@ -227,9 +232,11 @@ __device__ __forceinline__ float tile_make_p(const uint32_t* sr, uint32_t t_s, c
         }
         tmem_st16(t_s + c * 16, pk);
     }
-    float a, b;
-    unpack2(ls2, a, b);
-    return a + b;
+    xmax = fmaxf(xm[0], xm[1]);
+    float a, b, c, d;
+    unpack2(add2(ls2[0], ls2[1]), a, b);
+    unpack2(add2(ls2[2], ls2[3]), c, d);
+    return (a + b) + (c + d);
 }
 
 __device__ __forceinline__ void reg_dealloc_56() { asm volatile("setmaxnreg.dec.sync.aligned.u32 56;"); }
@@ -444,8 +451,9 @@ attend_kernel(const __grid_constant__ AttendParams p, const __grid_constant__ CU
             ve = max(127 - 60, min(127 + 60, ve));
             const float log2_sv = (float)(ve - 127);
 
-            float m = -INFINITY;   // running max of s * scale_k (lazy)
-            float l = 0.f;         // running sum of p / Sv
+            float m = 0.f;         // running max of s * scale_k (lazy; set by KV tile 0)
+            float l = 0.f;         // running sum of p / Sv, relative to m
+            float o_scale = 1.f;   // factor O still owes (applied before the next PV)
             const uint64_t c2c2 = pack2(c2, c2);
             const bool pingpong = n_qt == 2;
             int arrived = 0;       // KV tiles whose turn-barrier arrival this warpgroup has made
@@ -461,21 +469,44 @@ attend_kernel(const __grid_constant__ AttendParams p, const __grid_constant__ CU
 #pragma unroll
                 for (int c = 0; c < kBN / 32; ++c) tmem_ld32(t_s + c * 32, sr + c * 32);
                 tc_wait_ld();
-                // pass 1: u = s * scale_k and the row max over the valid keys
-                const float mt = nv == kBN ? tile_row_max<false>(sr, sm.sk[st], nv)
-                                           : tile_row_max<true>(sr, sm.sk[st], nv);
-                const float m_new = fmaxf(m, mt);
-                if (j == 0) {
-                    m = m_new;   // first tile: O not yet written
-                } else if (__any_sync(0xffffffffu, (m_new - m) * c2 > kLazyRescaleLog2)) {
-                    // Warp-uniform decision (the wait and the TMEM load/store
-                    // below are warp-collective); every lane moves to its own
-                    // new max (alpha = 1 where it did not grow).  O_t holds PV
-                    // up to tile j-1: wait for it to complete, scale in place.
+                if (j == 0)   // the first tile sets the reference max
+                    m = nv == kBN ? tile_row_max<false>(sr, sm.sk[st], nv)
+                                  : tile_row_max<true>(sr, sm.sk[st], nv);
+                // The warpgroups take turns on their exp passes (tile 0 of KV
+                // tile j, tile 1 of j, tile 0 of j+1, ...) through two named
+                // barriers; the waiting warpgroup is blocked in hardware.
+                if (pingpong && (t == 1 || j > 0)) named_bar_sync(t == 0 ? kBarTurn0 : kBarTurn1, 256);
+                // single pass against the running max: p/Sv = 2^(u*c2 - m*c2 - log2 Sv).
+                // If the tile outgrew the running max by more than f16 P holds,
+                // the pass is redone once against the tile's exact max (rare:
+                // the first tiles of a row).
+                float ls = 0.f, emax = 0.f;
+#pragma unroll 1
+                for (int attempt = 0; attempt < 2; ++attempt) {
+                    const float neg = -(m * c2 + log2_sv);
+                    float xmax;
+                    ls = nv == kBN
+                             ? tile_exp<false>(sr, t_s, sm.sk[st], sm.sv[st], c2c2, pack2(neg, neg), nv, xmax)
+                             : tile_exp<true>(sr, t_s, sm.sk[st], sm.sv[st], c2c2, pack2(neg, neg), nv, xmax);
+                    emax = xmax + log2_sv;   // max of (u - m) * c2 over the tile
+                    if (attempt == 1 || !__any_sync(0xffffffffu, emax > kRedoLog2)) break;
+                    const float mt = nv == kBN ? tile_row_max<false>(sr, sm.sk[st], nv)
+                                               : tile_row_max<true>(sr, sm.sk[st], nv);
+                    const float m_new = fmaxf(m, mt);
                     const float alpha = ex2((m - m_new) * c2);
                     l *= alpha;
+                    o_scale *= alpha;
                     m = m_new;
-                    if (!warp_wait(&sm.pv_done[t][(j - 1) & 1], ((j - 1) >> 1) & 1, limit)) { fail = true; break; }
+                    tc_wait_st();   // the first pass's P stores land before they are overwritten
+                }
+                l += ls;
+                if (pingpong && (t == 0 || j + 1 < n_tiles)) named_bar_arrive(t == 0 ? kBarTurn1 : kBarTurn0, 256);
+                arrived = j + 1;
+                // O owes a factor from an earlier move of m: apply it once PV(j-1)
+                // has completed and before PV(j) is issued (warp-uniform: the
+                // wait and the TMEM load/store are warp-collective).
+                if (__any_sync(0xffffffffu, o_scale != 1.f)) {
+                    if (j > 0 && !warp_wait(&sm.pv_done[t][(j - 1) & 1], ((j - 1) >> 1) & 1, limit)) { fail = true; break; }
                     tc_fence_after();
 #pragma unroll 1
                     for (int c = 0; c < D / 32; ++c) {
@@ -483,26 +514,22 @@ attend_kernel(const __grid_constant__ AttendParams p, const __grid_constant__ CU
                         tmem_ld32(t_o + c * 32, o);
                         tc_wait_ld();
 #pragma unroll
-                        for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+                        for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * o_scale);
                         tmem_st32(t_o + c * 32, o);
                     }
+                    o_scale = 1.f;
                 }
-                // pass 2: p / Sv = 2^(u*c2 - m*c2 - log2 Sv); P = (p / Sv) * scale_v.
-                // With two query tiles the warpgroups take turns (tile 0 of KV
-                // tile j, tile 1 of j, tile 0 of j+1, ...) through two named
-                // barriers: each exp phase runs with the exp unit to itself,
-                // and the waiting warpgroup is blocked in hardware, taking no
-                // issue slots from the one computing.
-                if (pingpong && (t == 1 || j > 0)) named_bar_sync(t == 0 ? kBarTurn0 : kBarTurn1, 256);
-                const float neg = -(m * c2 + log2_sv);
-                const uint64_t neg2 = pack2(neg, neg);
-                l += nv == kBN ? tile_make_p<false>(sr, t_s, sm.sv[st], c2c2, neg2, nv)
-                               : tile_make_p<true>(sr, t_s, sm.sv[st], c2c2, neg2, nv);
-                if (pingpong && (t == 0 || j + 1 < n_tiles)) named_bar_arrive(t == 0 ? kBarTurn1 : kBarTurn0, 256);
-                arrived = j + 1;
                 tc_wait_st();
                 tc_fence_before();
                 mbar_arrive(&sm.p_ready[t][b]);
+                // lazy move of the running max: only when this tile's scores grew
+                // past 2^8 of it; l now, O before the next PV (after PV(j)).
+                if (emax > kLazyRescaleLog2) {
+                    const float alpha = ex2(-emax);
+                    l *= alpha;
+                    o_scale *= alpha;
+                    m += emax / c2;
+                }
             }
             // On failure (which can only happen before a tile's turn sync),
             // still contribute to every remaining generation of both turn
@@ -518,7 +545,7 @@ attend_kernel(const __grid_constant__ AttendParams p, const __grid_constant__ CU
                 fail = true;
             if (!fail) {
                 tc_fence_after();
-                const float norm = 1.f / l;
+                const float norm = o_scale / l;
 #pragma unroll 1
                 for (int c = 0; c < D / 32; ++c) {
                     uint32_t o[32];
