@@ -28,8 +28,9 @@
 //              by more than 2^8.  The two warpgroups take turns on their exp
 //              phases, so each runs with the exp unit (16/clk/SM) to itself.
 // TMEM columns: S_t,b at 64*(2t+b) (64 columns each), O_0 [256,256+D),
-// O_1 [384,384+D).  QK(j+2) overwrites S_t,b only after PV(j), which reads
-// P_t,b out of it, has completed.
+// O_1 [384,384+D).  QK(j+2) overwrites S_t,b right after PV(j), which reads
+// P_t,b out of it, is issued: tcgen05 MMAs from one issuing thread execute in
+// order, so the write cannot overtake the read.
 //
 // Logical-to-physical frame order is resolved in the TMA coordinates: the
 // kernel receives the key set as a list of ring slots -- no gather, no copy.
@@ -376,11 +377,10 @@ attend_kernel(const __grid_constant__ AttendParams p, const __grid_constant__ CU
                     tc_commit(&sm.pv_done[t][b]);
                     tc_commit(&sm.kv_empty[j % kStages]);
                     tc_commit(&sm.tile_done[vb]);
-                    // S_t,b is free again once PV(j) has read P out of it
-                    if (j + 2 < n_tiles) {
-                        if (!mbar_wait_backoff(&sm.pv_done[t][b], (j >> 1) & 1, limit)) { fail = true; break; }
-                        if (!issue_qk(j + 2)) { fail = true; break; }
-                    }
+                    // QK(j+2) reuses S_t,b right behind PV(j), which reads P out of
+                    // it: tcgen05 MMAs issued by one thread execute in issue order,
+                    // so no completion wait is needed between them.
+                    if (j + 2 < n_tiles && !issue_qk(j + 2)) { fail = true; break; }
                 }
                 // drain: all MMAs issued by this thread complete before TMEM is freed
                 tc_commit(&sm.drain[t]);
