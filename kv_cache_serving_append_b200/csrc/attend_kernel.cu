@@ -10,7 +10,7 @@
 // definition, stated in rtv.h.
 //
 // One CTA = two 128-row query tiles of one head, sharing every K/V tile it
-// loads; KV tiles of 64 keys; 16 warps:
+// loads; KV tiles of 64 keys; 12 warps:
 //   warp 0     TMA producer: both Q tiles once; per KV tile the K and V code
 //              tiles at (ring slot * H + head, token tile) and their scales.
 //   warps 1,3  MMA issuers, one per query tile t (warp 1 also owns TMEM).
@@ -19,18 +19,14 @@
 //              (kind::f16, P read from TMEM where it overwrote S_t,b, V16
 //              from shared memory).  With two S buffers the softmax of KV tile
 //              j+1 runs while PV(j) and QK(j+2) execute.
-//   warps 4-7  widen the V code tile to f16 (exact) in the MN-major layout
-//              the PV MMA reads, a quarter each, one warp per SM sub-partition
-//              (one sub-partition's E4M3->f16 convert unit alone would pace
-//              the whole pipeline).  Warp 2 is idle.
-//   warps 8-11 softmax of query tile 0, warps 12-15 of query tile 1; one
-//              query row per thread, the tile's 64 scores in registers, one
-//              pass per KV tile against the running max: s*scale_k, exp2, row
-//              sum, P = p*scale_v/Sv in f16 written back over S; the tile max
-//              comes out of the same pass (a tile is redone against its exact
-//              max only when its p would leave f16 range); O is rescaled,
-//              lazily, only when the running max grows by more than 2^8.  The
-//              two warpgroups take turns on their exp passes.
+//   warp 2     widens the V code tile to f16 (exact) in the MN-major layout
+//              the PV MMA reads.
+//   warps 4-7  softmax of query tile 0, warps 8-11 of query tile 1; one query
+//              row per thread, the tile's 64 scores in registers: s*scale_k,
+//              running max, exp2, row sum, P = p*scale_v/Sv in f16 written
+//              back over S; lazy O rescaling only when the running max grows
+//              by more than 2^8.  The two warpgroups take turns on their exp
+//              phases, so each runs with the exp unit (16/clk/SM) to itself.
 // TMEM columns: S_t,b at 64*(2t+b) (64 columns each), O_0 [256,256+D),
 // O_1 [384,384+D).  QK(j+2) overwrites S_t,b right after PV(j), which reads
 // P_t,b out of it, is issued: tcgen05 MMAs from one issuing thread execute in
@@ -45,9 +41,9 @@
 // p*scale_v/Sv stays <= 2^8 inside f16 range, and 1/Sv is folded into the
 // exponent so the row sum carries the same factor and O/l needs none.
 //
-// Registers: the block launches with 128 per thread; the eight single-role
+// Registers: the block launches with 168 per thread; the four single-role
 // warps give theirs back (setmaxnreg 56) and the softmax warps take them
-// (setmaxnreg 200): 256 x 56 + 256 x 200 = 512 x 128.
+// (setmaxnreg 224): 128 x 56 + 256 x 224 = 384 x 168.
 //
 // Every mbarrier wait is bounded; on time-out a thread sets the error word,
 // leaves its loop, and the CTA drains its own async work before returning.
@@ -68,7 +64,7 @@ constexpr int kQT = 2;             // query tiles per CTA
 constexpr int kBN = kAttendKeys;   // keys per KV tile
 constexpr int kStages = 6;         // K/V code tile stages
 constexpr int kNV16 = 4;           // f16 V tile buffers
-constexpr int kThreads = 512;
+constexpr int kThreads = 384;
 constexpr uint32_t kTmemCols = 512;
 constexpr float kLazyRescaleLog2 = 8.0f;   // move the running max when a tile's p grows past 2^8
 constexpr float kRedoLog2 = 15.0f;         // redo a tile whose p would exceed 2^15 (f16 P range)
@@ -154,9 +150,9 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, long l
 {
     return __all_sync(0xffffffffu, mbar_wait(bar, parity, limit));
 }
-__device__ __forceinline__ bool warp_wait_backoff(uint64_t* bar, uint32_t parity, long long limit)
+__device__ __forceinline__ bool warp_wait_sleep(uint64_t* bar, uint32_t parity, long long limit)
 {
-    return __all_sync(0xffffffffu, mbar_wait_backoff(bar, parity, limit));
+    return __all_sync(0xffffffffu, mbar_wait_sleep(bar, parity, limit));
 }
 
 // Row max of u = s * scale_k over the valid keys of a KV tile (the kBN scores
@@ -245,7 +241,7 @@ __device__ __forceinline__ float tile_exp(const uint32_t* sr, uint32_t t_s, cons
 }
 
 __device__ __forceinline__ void reg_dealloc_56() { asm volatile("setmaxnreg.dec.sync.aligned.u32 56;"); }
-__device__ __forceinline__ void reg_alloc_200() { asm volatile("setmaxnreg.inc.sync.aligned.u32 200;"); }
+__device__ __forceinline__ void reg_alloc_224() { asm volatile("setmaxnreg.inc.sync.aligned.u32 224;"); }
 
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -284,7 +280,7 @@ attend_kernel(const __grid_constant__ AttendParams p, const __grid_constant__ CU
             mbar_init(&sm.drain[t], 1);
         }
         for (int b = 0; b < kNV16; ++b) {
-            mbar_init(&sm.v16_ready[b], 128);
+            mbar_init(&sm.v16_ready[b], 32);
             mbar_init(&sm.tile_done[b], n_qt);
         }
         fence_mbar_init();
@@ -306,10 +302,10 @@ attend_kernel(const __grid_constant__ AttendParams p, const __grid_constant__ CU
     const uint32_t tmem = sm.tmem_base;
     bool fail = false;
 
-    // setmaxnreg is executed by whole warpgroups (warps 0-3, 4-7, 8-11, 12-15),
-    // as the first instruction of each warpgroup's branch, so every region is
+    // setmaxnreg is executed by whole warpgroups (warps 0-3, 4-7, 8-11), as the
+    // first instruction of each warpgroup's branch, so every region is
     // allocated by ptxas under the budget it runs with.
-    if (warp < 8) {
+    if (warp < 4) {
         reg_dealloc_56();
         if (warp == 0) {
             // ------------------------------------------------------ producer --
@@ -390,24 +386,23 @@ attend_kernel(const __grid_constant__ AttendParams p, const __grid_constant__ CU
                 tc_commit(&sm.drain[t]);
                 if (!mbar_wait_backoff(&sm.drain[t], 0, limit)) fail = true;
             }
-        } else if (warp >= 4) {
+        } else if (warp == 2) {
             // ------------------------------------------- V widening (FP8->f16) --
             // A warp step covers 8 consecutive key rows x 4 chunk columns of one
             // 64-element block: in every 8-lane shared-memory phase the 8 rows hit
             // 8 different 16-byte bank groups, for the swizzled reads and for both
             // swizzled writes.
             constexpr int kNB = D / 64;                 // 64-element blocks per key row
-            const int cw = warp - 4;                    // widening warp 0..3, one per SM sub-partition
             const int rl = lane & 7, cq = lane >> 3;
             for (int j = 0; j < n_tiles; ++j) {
                 const int st = j % kStages, b = j % kNV16;
-                if (!warp_wait_backoff(&sm.k_full[st], (j / kStages) & 1, limit)) { fail = true; break; }
+                if (!warp_wait_sleep(&sm.k_full[st], (j / kStages) & 1, limit)) { fail = true; break; }
                 if (j >= kNV16 &&
-                    !warp_wait_backoff(&sm.tile_done[b], ((j / kNV16) - 1) & 1, limit)) { fail = true; break; }
+                    !warp_wait_sleep(&sm.tile_done[b], ((j / kNV16) - 1) & 1, limit)) { fail = true; break; }
                 const uint8_t* src = sm.v8[st];
                 uint8_t* dst = sm.v16[b];
     #pragma unroll 4
-                for (int combo = cw; combo < (kBN / 8) * kNB; combo += 4) {
+                for (int combo = 0; combo < (kBN / 8) * kNB; ++combo) {
                     const int r = (combo / kNB) * 8 + rl;
                     const int nb = combo % kNB;
                     const int c = nb * 4 + cq;                              // 16-byte chunk of the FP8 row
@@ -431,8 +426,8 @@ attend_kernel(const __grid_constant__ AttendParams p, const __grid_constant__ CU
         }
     } else {
         // --------------------------------------------------------- softmax --
-        reg_alloc_200();
-        const int t = (warp - 8) >> 2;              // query tile of this warpgroup
+        reg_alloc_224();
+        const int t = (warp - 4) >> 2;              // query tile of this warpgroup
         if (t < n_qt) {
             const int row = (warp & 3) * 32 + lane;     // TMEM lane == query row in tile
             const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
