@@ -22,11 +22,14 @@
 //   warp 2     widens the V code tile to f16 (exact) in the MN-major layout
 //              the PV MMA reads.
 //   warps 4-7  softmax of query tile 0, warps 8-11 of query tile 1; one query
-//              row per thread, the tile's 64 scores in registers: s*scale_k,
-//              running max, exp2, row sum, P = p*scale_v/Sv in f16 written
-//              back over S; lazy O rescaling only when the running max grows
-//              by more than 2^8.  The two warpgroups take turns on their exp
-//              phases, so each runs with the exp unit (16/clk/SM) to itself.
+//              row per thread, the tile's 64 scores in registers, one pass
+//              per KV tile against a reference m: s*scale_k, exp2, row sum,
+//              P = p*scale_v/Sv in f16 written back over S.  The row sum
+//              bounds every p of the tile, so it alone decides (no per-key
+//              max): a tile is redone against its exact max only when a row
+//              sum reaches 2^15 (f16 P range), and m moves up by a power of
+//              two, with O rescaled lazily, only when a row sum reaches 2^8.
+//              The two warpgroups run concurrently.
 // TMEM columns: S_t,b at 64*(2t+b) (64 columns each), O_0 [256,256+D),
 // O_1 [384,384+D).  QK(j+2) overwrites S_t,b right after PV(j), which reads
 // P_t,b out of it, is issued: tcgen05 MMAs from one issuing thread execute in
@@ -66,9 +69,8 @@ constexpr int kStages = 6;         // K/V code tile stages
 constexpr int kNV16 = 4;           // f16 V tile buffers
 constexpr int kThreads = 384;
 constexpr uint32_t kTmemCols = 512;
-constexpr float kLazyRescaleLog2 = 8.0f;   // move the running max when a tile's p grows past 2^8
-constexpr float kRedoLog2 = 15.0f;         // redo a tile whose p would exceed 2^15 (f16 P range)
-constexpr uint32_t kBarTurn0 = 1, kBarTurn1 = 2;   // named barriers: warpgroup 0 / 1 may start its exp phase
+constexpr int kLazyRescaleLog2 = 8;     // move the reference when a tile's row sum reaches 2^8 of it
+constexpr int kRedoLog2 = 15;           // redo a tile whose row sum reaches 2^15 (f16 P range)
 
 __host__ __device__ constexpr uint32_t col_s(int t, int b) { return 64u * (2 * t + b); }
 __host__ __device__ constexpr uint32_t col_o(int t) { return 256u + 128u * t; }
@@ -188,21 +190,19 @@ __device__ __forceinline__ float tile_row_max(const uint32_t* sr, const float* s
 }
 
 // One pass over a KV tile (the kBN scores of this thread's row in registers):
-// u = s * scale_k, x = u*c2 + neg (= (u - m)*c2 - log2 Sv for the running max
+// u = s * scale_k, x = u*c2 + neg (= (u - m)*c2 - log2 Sv for the reference
 // m), p/Sv = 2^x, P = (p/Sv) * scale_v packed to f16 pairs and written over S
 // in TMEM (keys [32c, 32c+32) -> P columns [16c, 16c+16); S is already in
-// registers).  Returns the row sum of p/Sv; xmax = max of x over valid keys,
-// from which the caller sees whether the tile outgrew the running max.
+// registers).  Returns the row sum of p/Sv, which also bounds every p/Sv of
+// the tile: the caller reads from it whether the tile outgrew m.
 template <bool kMask>
 __device__ __forceinline__ float tile_exp(const uint32_t* sr, uint32_t t_s, const float* sk,
-                                          const float* sv, uint64_t c2c2, uint64_t neg2, int nv,
-                                          float& xmax)
+                                          const float* sv, uint64_t c2c2, uint64_t neg2, int nv)
 {
     const float4* sk4 = reinterpret_cast<const float4*>(sk);
     const float4* sv4 = reinterpret_cast<const float4*>(sv);
-    // independent partial row sums and maxima: short dependency chains
+    // independent partial row sums: short dependency chains
     uint64_t ls2[4] = {pack2(0.f, 0.f), pack2(0.f, 0.f), pack2(0.f, 0.f), pack2(0.f, 0.f)};
-    float xm[2] = {-INFINITY, -INFINITY};
 #pragma unroll
     for (int c = 0; c < kBN / 32; ++c) {
         uint32_t pk[16];
@@ -221,7 +221,6 @@ __device__ __forceinline__ float tile_exp(const uint32_t* sr, uint32_t t_s, cons
                     if (k >= nv) x0 = -INFINITY;
                     if (k + 1 >= nv) x1 = -INFINITY;
                 }
-                xm[hh] = max3(xm[hh], x0, x1);
                 const float p0 = ex2(x0), p1 = ex2(x1);   // ex2(-inf) = 0 for masked keys
                 const uint64_t pp = pack2(p0, p1);
                 ls2[(k >> 1) & 3] = add2(ls2[(k >> 1) & 3], pp);
@@ -233,7 +232,6 @@ __device__ __forceinline__ float tile_exp(const uint32_t* sr, uint32_t t_s, cons
         }
         tmem_st16(t_s + c * 16, pk);
     }
-    xmax = fmaxf(xm[0], xm[1]);
     float a, b, c, d;
     unpack2(add2(ls2[0], ls2[1]), a, b);
     unpack2(add2(ls2[2], ls2[3]), c, d);
@@ -451,12 +449,11 @@ attend_kernel(const __grid_constant__ AttendParams p, const __grid_constant__ CU
             ve = max(127 - 60, min(127 + 60, ve));
             const float log2_sv = (float)(ve - 127);
 
-            float m = 0.f;         // running max of s * scale_k (lazy; set by KV tile 0)
+            float m = 0.f;         // reference of s * scale_k (the max of KV tile 0, moved up lazily)
             float l = 0.f;         // running sum of p / Sv, relative to m
             float o_scale = 1.f;   // factor O still owes (applied before the next PV)
             const uint64_t c2c2 = pack2(c2, c2);
-            const bool pingpong = n_qt == 2;
-            int arrived = 0;       // KV tiles whose turn-barrier arrival this warpgroup has made
+            const int log2_sv_i = ve - 127;
             for (int j = 0; j < n_tiles && !fail; ++j) {
                 const int st = j % kStages, b = j & 1;
                 const int fi = j / p.tiles_per_frame;
@@ -469,27 +466,24 @@ attend_kernel(const __grid_constant__ AttendParams p, const __grid_constant__ CU
 #pragma unroll
                 for (int c = 0; c < kBN / 32; ++c) tmem_ld32(t_s + c * 32, sr + c * 32);
                 tc_wait_ld();
-                if (j == 0)   // the first tile sets the reference max
+                if (j == 0)   // the first tile sets the reference
                     m = nv == kBN ? tile_row_max<false>(sr, sm.sk[st], nv)
                                   : tile_row_max<true>(sr, sm.sk[st], nv);
-                // The warpgroups take turns on their exp passes (tile 0 of KV
-                // tile j, tile 1 of j, tile 0 of j+1, ...) through two named
-                // barriers; the waiting warpgroup is blocked in hardware.
-                if (pingpong && (t == 1 || j > 0)) named_bar_sync(t == 0 ? kBarTurn0 : kBarTurn1, 256);
-                // single pass against the running max: p/Sv = 2^(u*c2 - m*c2 - log2 Sv).
-                // If the tile outgrew the running max by more than f16 P holds,
-                // the pass is redone once against the tile's exact max (rare:
-                // the first tiles of a row).
-                float ls = 0.f, emax = 0.f;
+                // single pass against the reference: p/Sv = 2^(u*c2 - m*c2 - log2 Sv).
+                // The row sum bounds every p of the tile; if some row's sum
+                // (times Sv) reaches 2^15, a p may be past f16 P range and the
+                // pass is redone once against the tile's exact max (rare: the
+                // first tiles of a row).  ls_e = floor(log2(row sum * Sv)).
+                float ls = 0.f;
+                int ls_e = 0;
 #pragma unroll 1
                 for (int attempt = 0; attempt < 2; ++attempt) {
                     const float neg = -(m * c2 + log2_sv);
-                    float xmax;
                     ls = nv == kBN
-                             ? tile_exp<false>(sr, t_s, sm.sk[st], sm.sv[st], c2c2, pack2(neg, neg), nv, xmax)
-                             : tile_exp<true>(sr, t_s, sm.sk[st], sm.sv[st], c2c2, pack2(neg, neg), nv, xmax);
-                    emax = xmax + log2_sv;   // max of (u - m) * c2 over the tile
-                    if (attempt == 1 || !__any_sync(0xffffffffu, emax > kRedoLog2)) break;
+                             ? tile_exp<false>(sr, t_s, sm.sk[st], sm.sv[st], c2c2, pack2(neg, neg), nv)
+                             : tile_exp<true>(sr, t_s, sm.sk[st], sm.sv[st], c2c2, pack2(neg, neg), nv);
+                    ls_e = (int)((__float_as_uint(ls) >> 23) & 0xff) - 127 + log2_sv_i;
+                    if (attempt == 1 || !__any_sync(0xffffffffu, ls_e >= kRedoLog2)) break;
                     const float mt = nv == kBN ? tile_row_max<false>(sr, sm.sk[st], nv)
                                                : tile_row_max<true>(sr, sm.sk[st], nv);
                     const float m_new = fmaxf(m, mt);
@@ -500,8 +494,6 @@ attend_kernel(const __grid_constant__ AttendParams p, const __grid_constant__ CU
                     tc_wait_st();   // the first pass's P stores land before they are overwritten
                 }
                 l += ls;
-                if (pingpong && (t == 0 || j + 1 < n_tiles)) named_bar_arrive(t == 0 ? kBarTurn1 : kBarTurn0, 256);
-                arrived = j + 1;
                 // O owes a factor from an earlier move of m: apply it once PV(j-1)
                 // has completed and before PV(j) is issued (warp-uniform: the
                 // wait and the TMEM load/store are warp-collective).
@@ -522,25 +514,16 @@ attend_kernel(const __grid_constant__ AttendParams p, const __grid_constant__ CU
                 tc_wait_st();
                 tc_fence_before();
                 mbar_arrive(&sm.p_ready[t][b]);
-                // lazy move of the running max: only when this tile's scores grew
-                // past 2^8 of it; l now, O before the next PV (after PV(j)).
-                if (emax > kLazyRescaleLog2) {
-                    const float alpha = ex2(-emax);
+                // lazy move of the reference: only when this tile's row sum grew
+                // to 2^8 of it; by an exact power of two, l now, O before the next
+                // PV (after PV(j)).
+                if (ls_e >= kLazyRescaleLog2) {
+                    const float alpha = __uint_as_float((uint32_t)(127 - ls_e) << 23);   // 2^-ls_e
                     l *= alpha;
                     o_scale *= alpha;
-                    m += emax / c2;
+                    m += (float)ls_e / c2;
                 }
             }
-            // On failure (which can only happen before a tile's turn sync),
-            // still contribute to every remaining generation of both turn
-            // barriers -- an arrive in place of each sync, then the tile's own
-            // arrive -- so every barrier generation completes exactly as in a
-            // normal run and no warp can block in a named-barrier sync.
-            if (pingpong)
-                for (int j = arrived; j < n_tiles; ++j) {
-                    if (t == 1 || j > 0) named_bar_arrive(t == 0 ? kBarTurn0 : kBarTurn1, 256);
-                    if (t == 0 || j + 1 < n_tiles) named_bar_arrive(t == 0 ? kBarTurn1 : kBarTurn0, 256);
-                }
             if (!fail && !warp_wait(&sm.pv_done[t][(n_tiles - 1) & 1], ((n_tiles - 1) >> 1) & 1, limit))
                 fail = true;
             if (!fail) {
