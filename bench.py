@@ -333,6 +333,9 @@ def main():
         t = torch.tensor([elapsed_ms], device=dev, dtype=torch.float64)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         elapsed_ms = float(t.item())
+    # kernels per step: append, attention, and the split merge when the key range is split
+    splits = cache.state().last_attend_splits
+    launches_per_step = 2 + (1 if splits > 1 else 0)
     append_ms = statistics.mean(ev[i][0].elapsed_time(ev[i][1]) for i in range(args.steps))
     attend_ms = statistics.mean(ev[i][1].elapsed_time(ev[i][2]) for i in range(args.steps))
 
@@ -384,7 +387,7 @@ def main():
         "data": "synthetic", "config": config_block(cfg),
         "append_gbs": append_gbs, "append_us": append_ms * 1e3,
         "attn_tflops": attn_tflops, "attn_us": attend_ms * 1e3,
-        "roofline": {"kernel": "rtv attend (tcgen05 FP8 attention)", "bound": "tensor",
+        "roofline": {"kernel": "rtv attend (tcgen05 FP8 attention; with a split key range the timed call includes the merge kernel)", "bound": "tensor",
                      "achieved": attn_tflops, "peak": fp8_peak, "unit": "TFLOP/s",
                      "frac": attn_tflops / fp8_peak,
                      "peak_source": f"{peak_src} bf16 burst {bf16_tf} TFLOP/s x 2 (nominal "
@@ -398,7 +401,8 @@ def main():
                             "algorithmic_bytes_per_launch": wl["append_bytes"]},
         "e2e": {"value": e2e_ms * 1e3 / (e2e_steps * world), "unit": "us/layer-step",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-        "gpu_launches": 2 * args.steps,
+        "gpu_launches": launches_per_step * args.steps,
+        "attend_key_splits": splits,
         "clocks": clocks,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

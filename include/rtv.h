@@ -108,6 +108,10 @@ typedef struct {
  *   frame_of_slot        per slot, the visible frame it holds, or -1
  *   staged_layers        layers that currently hold staged frames
  *   staged_frames        their frame count (-1 if the layers disagree)
+ *   last_attend_splits   key-range splits of the last rtv_attend call (0
+ *                        before the first): 1 = one kernel, s > 1 = the
+ *                        attention kernel over s key ranges plus a merge
+ *                        kernel
  */
 typedef struct {
     long long frames_committed;
@@ -121,6 +125,7 @@ typedef struct {
     long long frame_of_slot[RTV_MAX_SLOTS];
     int staged_layers;
     int staged_frames;
+    int last_attend_splits;
 } rtv_cache_state;
 
 /*
@@ -143,8 +148,9 @@ const char* rtv_status_string(rtv_status status);
 
 /*
  * Device bytes a cache with this configuration needs (K/V rings, scales, Q
- * workspaces, RoPE tables, error word), so that a caller can allocate them
- * itself.  Errors: RTV_ERR_INVALID_ARG (NULL or inconsistent config),
+ * workspaces, RoPE tables, the key-range split partials of one attention
+ * call -- 4 x F_max*T x n_heads x (head_dim + 2) fp32, shared by all layers --
+ * and the error word), so that a caller can allocate them itself.  Errors: RTV_ERR_INVALID_ARG (NULL or inconsistent config),
  * RTV_ERR_UNSUPPORTED (head_dim or RoPE split the kernels do not implement).
  */
 rtv_status rtv_cache_required_bytes(const rtv_cache_config* cfg, size_t* bytes);
@@ -192,6 +198,13 @@ rtv_status rtv_cache_append(rtv_cache* cache, int layer, const void* q, const vo
  * One kernel: TMA loads of Q/K/V codes and scales by (slot, head, token
  * tile) coordinates, QK^T in FP8 E4M3 on tcgen05 tensor cores into TMEM,
  * online softmax in registers, PV on tcgen05 with P and the V codes in f16.
+ * When one CTA per (head, 256 query rows) would leave the GPU's last wave of
+ * CTAs mostly idle, the key set is split into up to 4 ranges (grid z): each
+ * CTA writes its range's unnormalised O and row statistics to the cache
+ * buffer's split section and a second kernel merges them (online-softmax
+ * merge) into out.  That section is shared by all layers: attention calls on
+ * one cache must be ordered on one stream (as the append/attend/advance
+ * sequence already is); overlapping calls race.
  * Errors: RTV_ERR_INVALID_ARG, RTV_ERR_STATE (layer has no staged frames),
  * RTV_ERR_CUDA.  A kernel timeout is reported by rtv_poll_error.
  */

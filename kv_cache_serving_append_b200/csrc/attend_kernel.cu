@@ -258,7 +258,9 @@ attend_kernel(const __grid_constant__ AttendParams p, const __grid_constant__ CU
     const int q0 = blockIdx.x * (kQT * kBM);
     const int h = blockIdx.y;
     const int H = p.H;
-    const int n_tiles = p.n_frames_keys * p.tiles_per_frame;
+    // this CTA's range of the key set: KV tiles [j0, j0 + n_tiles) (blockIdx.z = split)
+    const int j0 = blockIdx.z * p.tiles_per_split;
+    const int n_tiles = min(p.n_frames_keys * p.tiles_per_frame - j0, p.tiles_per_split);
     const int n_qt = min(kQT, (p.M - q0 + kBM - 1) / kBM);   // query tiles with valid rows
     const long long limit = p.wait_limit;
 
@@ -319,8 +321,8 @@ attend_kernel(const __grid_constant__ AttendParams p, const __grid_constant__ CU
                         fail = true;
                         break;
                     }
-                    const int fi = j / p.tiles_per_frame;
-                    const int t0 = (j - fi * p.tiles_per_frame) * kBN;
+                    const int fi = (j0 + j) / p.tiles_per_frame;
+                    const int t0 = (j0 + j - fi * p.tiles_per_frame) * kBN;
                     const int row = p.slot[fi] * H + h;
                     mbar_arrive_expect_tx(&sm.k_full[st], 2 * kKVBytes + 2 * kBN * 4);
                     tma_load_3d(sm.k[st], &map_k, &sm.k_full[st], 0, t0, row);
@@ -456,8 +458,8 @@ attend_kernel(const __grid_constant__ AttendParams p, const __grid_constant__ CU
             const int log2_sv_i = ve - 127;
             for (int j = 0; j < n_tiles && !fail; ++j) {
                 const int st = j % kStages, b = j & 1;
-                const int fi = j / p.tiles_per_frame;
-                const int nv = min(kBN, p.T - (j - fi * p.tiles_per_frame) * kBN);
+                const int fi = (j0 + j) / p.tiles_per_frame;
+                const int nv = min(kBN, p.T - (j0 + j - fi * p.tiles_per_frame) * kBN);
                 const uint32_t t_s = tmem + lane_off + col_s(t, b);
                 if (!warp_wait(&sm.k_full[st], (j / kStages) & 1, limit)) { fail = true; break; }
                 if (!warp_wait(&sm.s_full[t][b], (j >> 1) & 1, limit)) { fail = true; break; }
@@ -528,14 +530,22 @@ attend_kernel(const __grid_constant__ AttendParams p, const __grid_constant__ CU
                 fail = true;
             if (!fail) {
                 tc_fence_after();
-                const float norm = o_scale / l;
+                // one split: the normalised output.  Several: this range's O
+                // (owed factor applied, not normalised) and its row statistics
+                // (reference exponent m*c2, row sum l), merged by the combine
+                // kernel.
+                const bool split = p.n_split > 1;
+                const size_t part_row = ((size_t)blockIdx.z * p.M + qrow) * H + h;
+                if (split && row_ok)
+                    *reinterpret_cast<float2*>(p.part_ml + 2 * part_row) = make_float2(m * c2, l);
+                const float norm = split ? o_scale : o_scale / l;
 #pragma unroll 1
                 for (int c = 0; c < D / 32; ++c) {
                     uint32_t o[32];
                     tmem_ld32(t_o + c * 32, o);
                     tc_wait_ld();
                     if (row_ok) {
-                        if (p.out_bf16) {
+                        if (p.out_bf16 && !split) {
                             __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(p.out) +
                                                  ((size_t)qrow * H + h) * D + c * 32;
 #pragma unroll
@@ -551,7 +561,9 @@ attend_kernel(const __grid_constant__ AttendParams p, const __grid_constant__ CU
                                 *reinterpret_cast<uint4*>(dst + i) = make_uint4(w[0], w[1], w[2], w[3]);
                             }
                         } else {
-                            float* dst = reinterpret_cast<float*>(p.out) + ((size_t)qrow * H + h) * D + c * 32;
+                            float* dst = (split ? p.part_o + part_row * D
+                                                : reinterpret_cast<float*>(p.out) + ((size_t)qrow * H + h) * D) +
+                                         c * 32;
 #pragma unroll
                             for (int i = 0; i < 32; i += 4)
                                 *reinterpret_cast<float4*>(dst + i) = make_float4(
@@ -574,6 +586,48 @@ attend_kernel(const __grid_constant__ AttendParams p, const __grid_constant__ CU
     }
 }
 
+// Merge of the key-range splits: one warp per (query row, head).  Split s
+// holds O_s = sum_{keys in s} 2^(x - e_s) v (unnormalised) and l_s = sum 2^(x
+// - e_s) against its own reference exponent e_s; out = sum_s 2^(e_s - e) O_s
+// / sum_s 2^(e_s - e) l_s with e = max_s e_s (the online-softmax merge).
+template <int D>
+__global__ void __launch_bounds__(256) combine_kernel(const AttendParams p)
+{
+    const int warp = (blockIdx.x * 256 + threadIdx.x) >> 5;
+    const int lane = threadIdx.x & 31;
+    if (warp >= p.M * p.H) return;
+    const size_t stride = (size_t)p.M * p.H;          // rows of one split
+    float e = -INFINITY;
+    for (int s = 0; s < p.n_split; ++s) e = fmaxf(e, p.part_ml[2 * (s * stride + warp)]);
+    constexpr int kV = D / 32;                          // elements per lane
+    float acc[kV] = {};
+    float lsum = 0.f;
+    for (int s = 0; s < p.n_split; ++s) {
+        const float2 ml = *reinterpret_cast<const float2*>(p.part_ml + 2 * (s * stride + warp));
+        const float w = exp2f(ml.x - e);
+        lsum += w * ml.y;
+        const float* src = p.part_o + (s * stride + warp) * D + lane * kV;
+        if constexpr (kV == 4) {
+            const float4 v = *reinterpret_cast<const float4*>(src);
+            acc[0] += w * v.x; acc[1] += w * v.y; acc[2] += w * v.z; acc[3] += w * v.w;
+        } else {
+            const float2 v = *reinterpret_cast<const float2*>(src);
+            acc[0] += w * v.x; acc[1] += w * v.y;
+        }
+    }
+    const float inv = 1.f / lsum;
+    if (p.out_bf16) {
+        __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(p.out) + (size_t)warp * D + lane * kV;
+#pragma unroll
+        for (int i = 0; i < kV; i += 2)
+            *reinterpret_cast<__nv_bfloat162*>(dst + i) = __floats2bfloat162_rn(acc[i] * inv, acc[i + 1] * inv);
+    } else {
+        float* dst = reinterpret_cast<float*>(p.out) + (size_t)warp * D + lane * kV;
+#pragma unroll
+        for (int i = 0; i < kV; ++i) dst[i] = acc[i] * inv;
+    }
+}
+
 template <int D>
 cudaError_t launch(const AttendParams& p, const CUtensorMap* maps, cudaStream_t stream)
 {
@@ -587,8 +641,12 @@ cudaError_t launch(const AttendParams& p, const CUtensorMap* maps, cudaStream_t 
         if (e != cudaSuccess) return e;
         configured |= 1u << dev;
     }
-    dim3 grid((p.M + kQT * kBM - 1) / (kQT * kBM), p.H);
+    dim3 grid((p.M + kQT * kBM - 1) / (kQT * kBM), p.H, p.n_split);
     attend_kernel<D><<<grid, kThreads, smem, stream>>>(p, maps[0], maps[1], maps[2], maps[3], maps[4]);
+    if (p.n_split > 1) {
+        const long long warps = (long long)p.M * p.H;
+        combine_kernel<D><<<(unsigned)((warps + 7) / 8), 256, 0, stream>>>(p);
+    }
     return cudaGetLastError();
 }
 

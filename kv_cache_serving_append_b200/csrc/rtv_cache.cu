@@ -34,6 +34,10 @@ struct rtv_cache {
     float* h_table = nullptr;
     float* w_table = nullptr;
     unsigned int* err = nullptr;
+    float* part_o = nullptr;            // key-range split partials of one attention call
+    float* part_ml = nullptr;
+    int sm_count = 148;
+    int last_splits = 0;
     // ring state
     long long G = 0;
     bool pinned_committed = false;
@@ -80,7 +84,7 @@ rtv_status validate(const rtv_cache_config* c)
 
 struct Geometry {
     int T, S, q_rows, scale_pitch, q_scale_pitch;
-    size_t layer_bytes, tables_off, err_off, total;
+    size_t layer_bytes, tables_off, split_o_off, split_ml_off, err_off, total;
     rtv_layer_layout rel;   // offsets relative to the layer base
 };
 
@@ -106,7 +110,12 @@ Geometry geometry(const rtv_cache_config* c)
     g.layer_bytes = off;
     g.tables_off = g.layer_bytes * c->n_layers;
     const size_t table_bytes = ((size_t)c->grid_h * c->rope_h + (size_t)c->grid_w * c->rope_w) * 4;
-    g.err_off = align_up(g.tables_off + table_bytes, kAlign);
+    // partials of the key-range splits: [kMaxSplit][q_rows][H][D] O, then
+    // [kMaxSplit][q_rows][H][2] statistics (shared by all layers: one call at a time)
+    const size_t split_rows = (size_t)kMaxSplit * g.q_rows * c->n_heads;
+    g.split_o_off = align_up(g.tables_off + table_bytes, kAlign);
+    g.split_ml_off = align_up(g.split_o_off + split_rows * c->head_dim * 4, kAlign);
+    g.err_off = align_up(g.split_ml_off + split_rows * 2 * 4, kAlign);
     g.total = align_up(g.err_off + 256, kAlign);
     return g;
 }
@@ -292,6 +301,15 @@ rtv_status rtv_cache_create(const rtv_cache_config* cfg, void* device_buf, size_
     c->h_table = reinterpret_cast<float*>(c->buf + g.tables_off);
     c->w_table = c->h_table + (size_t)cfg->grid_h * cfg->rope_h;
     c->err = reinterpret_cast<unsigned int*>(c->buf + g.err_off);
+    c->part_o = reinterpret_cast<float*>(c->buf + g.split_o_off);
+    c->part_ml = reinterpret_cast<float*>(c->buf + g.split_ml_off);
+    {
+        int sms = 0;
+        if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, c->device) == cudaSuccess && sms > 0)
+            c->sm_count = sms;
+        else
+            cudaGetLastError();
+    }
     c->staged.assign(cfg->n_layers, 0);
     c->frame_of_slot.assign(c->S, -1);
 
@@ -403,6 +421,27 @@ rtv_status rtv_attend(rtv_cache* c, int layer, void* out, int out_dtype, void* s
     for (int s : c->visible_slots) p.slot[nk++] = s;
     for (int f = 0; f < n; ++f) p.slot[nk++] = staged_slot(c, f);
     p.n_frames_keys = nk;
+    // Key-range splits: one CTA per (head, 256 query rows) alone gives
+    // ceil(units / SMs) waves of equal CTAs; splitting every unit's key range
+    // s ways fills the last wave better at the price of a merge pass.  Pick s
+    // with the least ceil(units * s / SMs) / s, charging 3% of a full-range
+    // CTA per extra split (pipeline fill and drain, partial write and merge),
+    // and keep at least 8 KV tiles per split.
+    const int units = ((p.M + 2 * kAttendRows - 1) / (2 * kAttendRows)) * p.H;
+    const int n_all = nk * p.tiles_per_frame;
+    int best_s = 1;
+    double best_cost = 1e30;
+    for (int s = 1; s <= kMaxSplit; ++s) {
+        if (s > 1 && n_all / s < 8) break;
+        const long long waves = ((long long)units * s + c->sm_count - 1) / c->sm_count;
+        const double cost = (double)waves / s + 0.03 * (s - 1);
+        if (cost < best_cost - 1e-9) { best_cost = cost; best_s = s; }
+    }
+    p.tiles_per_split = (n_all + best_s - 1) / best_s;
+    p.n_split = (n_all + p.tiles_per_split - 1) / p.tiles_per_split;   // no empty split
+    p.part_o = c->part_o;
+    p.part_ml = c->part_ml;
+    c->last_splits = p.n_split;
     p.debug_wait_fault = c->debug_wait_fault;
     p.wait_limit = c->wait_limit;
     c->debug_wait_fault = 0;
@@ -466,6 +505,7 @@ rtv_status rtv_cache_get_state(const rtv_cache* c, rtv_cache_state* out)
         }
     out->staged_layers = ns;
     out->staged_frames = nf;
+    out->last_attend_splits = c->last_splits;
     return RTV_OK;
 }
 

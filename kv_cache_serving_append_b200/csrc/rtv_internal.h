@@ -19,6 +19,7 @@ constexpr int kMaxRopeHalf = 32;   // rope_t / 2 <= 32 (frame-axis table travels
 // 128 query rows per query tile, 64 keys per KV tile.
 constexpr int kAttendRows = 128;
 constexpr int kAttendKeys = 64;
+constexpr int kMaxSplit = 4;       // key-range splits of one attention call
 
 // Device error word bits.
 constexpr uint32_t kErrTimeout = 1u;
@@ -55,6 +56,10 @@ struct AttendParams {
     int out_bf16;
     int n_frames_keys;             // frames in the key set
     int tiles_per_frame;           // ceil(T / kAttendKeys)
+    int n_split;                   // key-range splits (grid z); 1: no partials
+    int tiles_per_split;           // KV tiles per split (the last may hold fewer)
+    float* part_o;                 // [n_split][M][H][D] unnormalised O per split
+    float* part_ml;                // [n_split][M][H][2] (reference exponent, row sum)
     int debug_wait_fault;          // 1: producer never arms the first barrier
     long long wait_limit;          // per-wait limit in clock cycles
     int slot[kMaxSlots];           // key set, logical order

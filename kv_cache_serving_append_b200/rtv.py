@@ -43,7 +43,8 @@ class rtv_cache_state(ctypes.Structure):
                 ("visible_slots", ctypes.c_int * RTV_MAX_SLOTS),
                 ("visible_frames", ctypes.c_longlong * RTV_MAX_SLOTS),
                 ("frame_of_slot", ctypes.c_longlong * RTV_MAX_SLOTS),
-                ("staged_layers", ctypes.c_int), ("staged_frames", ctypes.c_int)]
+                ("staged_layers", ctypes.c_int), ("staged_frames", ctypes.c_int),
+                ("last_attend_splits", ctypes.c_int)]
 
 
 class rtv_layer_layout(ctypes.Structure):
