@@ -202,6 +202,23 @@ class OracleTimer:
         return us, desc
 
 
+def max_over_ranks(value_ms: float, world: int, device) -> float:
+    """The slowest rank's time: every rank's timed region is reduced with MAX
+    (replicas: one independent cache per GPU, no data-path collective)."""
+    if world <= 1:
+        return value_ms
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value_ms], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def us_per_layer_step(elapsed_ms: float, steps: int, world: int) -> float:
+    """Whole-job figure: the max-over-ranks time over the layer-steps all ranks did."""
+    return elapsed_ms * 1e3 / (steps * world)
+
+
 def run_reference(args):
     """--impl reference: the CPU oracle as it stands, on the host cores."""
     rank = int(os.environ.get("RANK", "0"))
@@ -328,11 +345,7 @@ def main():
     clocks = sampler.stop() if sampler else None
     if cache.poll_error():
         raise RuntimeError("kernel error in the timed region")
-    elapsed_ms = t_start.elapsed_time(t_end)
-    if world > 1:
-        t = torch.tensor([elapsed_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        elapsed_ms = float(t.item())
+    elapsed_ms = max_over_ranks(t_start.elapsed_time(t_end), world, dev)
     # kernels per step: append, attention, and the split merge when the key range is split
     splits = cache.state().last_attend_splits
     launches_per_step = 2 + (1 if splits > 1 else 0)
@@ -366,11 +379,7 @@ def main():
         e2e_step(i)
     e1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1)
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
     h2d = sum(t.numel() * t.element_size() for t in dev_in)
     d2h = host_out.numel() * host_out.element_size()
 
@@ -378,7 +387,7 @@ def main():
     fp8_peak = 2.0 * bf16_tf
     attn_tflops = wl["flops"] / (attend_ms * 1e-3) / 1e12
     append_gbs = wl["append_bytes"] / (append_ms * 1e-3) / 1e9
-    us_per_step = elapsed_ms * 1e3 / (args.steps * world)
+    us_per_step = us_per_layer_step(elapsed_ms, args.steps, world)
     line = {
         "metric": METRIC, "value": us_per_step, "unit": "us/layer-step", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup,
