@@ -239,6 +239,26 @@ rtv_status rtv_cache_export(const rtv_cache* cache, int layer, int slot, void* c
 rtv_status rtv_poll_error(rtv_cache* cache);
 
 /*
+ * rtv_attend for callers that cannot allocate device memory: the same
+ * kernels and results (bit for bit), but the key-range split partials go to a
+ * fixed 16 MiB device array compiled into the library (file-scope
+ * __device__, its address looked up once per device) instead of the cache
+ * buffer's split section.  The call allocates nothing (no cudaMalloc/
+ * cudaFree, no allocating library routine).  Nothing in the array needs to
+ * start at zero: the merge reads only partials the same call wrote.  The array
+ * is shared by every cache and stream on the device: calls that overlap in
+ * time (other streams, other host threads) race.  A call whose split plan
+ * needs more than 16 MiB of partials (n_split x n_frames*T x n_heads x
+ * (head_dim + 2) fp32) is rejected with RTV_ERR_UNSUPPORTED before anything
+ * is launched; an unsplit call needs none.  The method's sources describe no
+ * counterpart of this entry point: it is a deployment convenience.
+ * Errors: as rtv_attend, plus RTV_ERR_UNSUPPORTED (partials over 16 MiB) and
+ * RTV_ERR_CUDA (symbol lookup failed).
+ */
+rtv_status rtv_attend_static_scratch(rtv_cache* cache, int layer, void* out, int out_dtype,
+                                     void* stream);
+
+/*
  * Test hook: when set to 1, the next rtv_attend launches the kernel in a mode
  * where its first wait can never complete (the producer never arms the
  * barrier and issues no copy), so every wait runs into its time limit, the

@@ -17,6 +17,7 @@
 #include <cstdlib>
 #include <cstring>
 #include <new>
+#include <mutex>
 #include <vector>
 
 #include "rtv_internal.h"
@@ -35,7 +36,6 @@ struct rtv_cache {
     float* w_table = nullptr;
     unsigned int* err = nullptr;
     float* part_o = nullptr;            // key-range split partials of one attention call
-    float* part_ml = nullptr;
     int sm_count = 148;
     int last_splits = 0;
     // ring state
@@ -84,7 +84,7 @@ rtv_status validate(const rtv_cache_config* c)
 
 struct Geometry {
     int T, S, q_rows, scale_pitch, q_scale_pitch;
-    size_t layer_bytes, tables_off, split_o_off, split_ml_off, err_off, total;
+    size_t layer_bytes, tables_off, split_off, err_off, total;
     rtv_layer_layout rel;   // offsets relative to the layer base
 };
 
@@ -110,12 +110,11 @@ Geometry geometry(const rtv_cache_config* c)
     g.layer_bytes = off;
     g.tables_off = g.layer_bytes * c->n_layers;
     const size_t table_bytes = ((size_t)c->grid_h * c->rope_h + (size_t)c->grid_w * c->rope_w) * 4;
-    // partials of the key-range splits: [kMaxSplit][q_rows][H][D] O, then
-    // [kMaxSplit][q_rows][H][2] statistics (shared by all layers: one call at a time)
+    // partials of the key-range splits, room for kMaxSplit x q_rows x H rows of
+    // D + 2 floats (O, then the statistics; shared by all layers: one call at a time)
     const size_t split_rows = (size_t)kMaxSplit * g.q_rows * c->n_heads;
-    g.split_o_off = align_up(g.tables_off + table_bytes, kAlign);
-    g.split_ml_off = align_up(g.split_o_off + split_rows * c->head_dim * 4, kAlign);
-    g.err_off = align_up(g.split_ml_off + split_rows * 2 * 4, kAlign);
+    g.split_off = align_up(g.tables_off + table_bytes, kAlign);
+    g.err_off = align_up(g.split_off + split_rows * (c->head_dim + 2) * 4, kAlign);
     g.total = align_up(g.err_off + 256, kAlign);
     return g;
 }
@@ -301,8 +300,7 @@ rtv_status rtv_cache_create(const rtv_cache_config* cfg, void* device_buf, size_
     c->h_table = reinterpret_cast<float*>(c->buf + g.tables_off);
     c->w_table = c->h_table + (size_t)cfg->grid_h * cfg->rope_h;
     c->err = reinterpret_cast<unsigned int*>(c->buf + g.err_off);
-    c->part_o = reinterpret_cast<float*>(c->buf + g.split_o_off);
-    c->part_ml = reinterpret_cast<float*>(c->buf + g.split_ml_off);
+    c->part_o = reinterpret_cast<float*>(c->buf + g.split_off);
     {
         int sms = 0;
         if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, c->device) == cudaSuccess && sms > 0)
@@ -397,7 +395,14 @@ rtv_status rtv_cache_append(rtv_cache* c, int layer, const void* q, const void* 
     return RTV_OK;
 }
 
-rtv_status rtv_attend(rtv_cache* c, int layer, void* out, int out_dtype, void* stream)
+namespace {
+
+// Attention launch shared by rtv_attend and rtv_attend_static_scratch.  The
+// split partials go to part_o / part_ml (capacity_bytes of room, in floats:
+// n_split*M*H*D of O, then n_split*M*H*2 of statistics); a plan whose
+// partials do not fit is rejected with RTV_ERR_UNSUPPORTED before any launch.
+rtv_status attend_impl(rtv_cache* c, int layer, void* out, int out_dtype, void* stream,
+                       float* part_base, size_t capacity_bytes)
 {
     if (!c || layer < 0 || layer >= c->cfg.n_layers) return RTV_ERR_INVALID_ARG;
     if (!out || !aligned16(out)) return RTV_ERR_INVALID_ARG;
@@ -439,16 +444,62 @@ rtv_status rtv_attend(rtv_cache* c, int layer, void* out, int out_dtype, void* s
     }
     p.tiles_per_split = (n_all + best_s - 1) / best_s;
     p.n_split = (n_all + p.tiles_per_split - 1) / p.tiles_per_split;   // no empty split
-    p.part_o = c->part_o;
-    p.part_ml = c->part_ml;
-    c->last_splits = p.n_split;
+    const size_t part_rows = (size_t)p.n_split * p.M * p.H;
+    if (p.n_split > 1 && part_rows * (p.D + 2) * sizeof(float) > capacity_bytes) return RTV_ERR_UNSUPPORTED;
+    p.part_o = part_base;
+    p.part_ml = part_base + part_rows * p.D;
     p.debug_wait_fault = c->debug_wait_fault;
     p.wait_limit = c->wait_limit;
     c->debug_wait_fault = 0;
+    c->last_splits = p.n_split;
     if (launch_attend(p, &c->maps[(size_t)layer * 5], c->D, static_cast<cudaStream_t>(stream)) !=
         cudaSuccess)
         return RTV_ERR_CUDA;
     return RTV_OK;
+}
+
+// Split partials of rtv_attend_static_scratch: a fixed device array (16 MiB),
+// shared by every cache and stream of the device.
+constexpr size_t kStaticScratchFloats = (size_t)4 << 20;
+__device__ __align__(256) float g_static_scratch[kStaticScratchFloats];
+
+// Address of g_static_scratch on the current device, looked up once per device.
+rtv_status static_scratch_address(int device, float** out)
+{
+    static std::mutex mu;
+    static void* addr[64] = {};
+    if (device < 0 || device >= 64) return RTV_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!addr[device]) {
+        void* a = nullptr;
+        if (cudaGetSymbolAddress(&a, g_static_scratch) != cudaSuccess || !a) {
+            cudaGetLastError();
+            return RTV_ERR_CUDA;
+        }
+        addr[device] = a;
+    }
+    *out = static_cast<float*>(addr[device]);
+    return RTV_OK;
+}
+
+}  // namespace
+
+rtv_status rtv_attend(rtv_cache* c, int layer, void* out, int out_dtype, void* stream)
+{
+    if (!c) return RTV_ERR_INVALID_ARG;
+    // the cache buffer's split section holds kMaxSplit * F_max*T * H rows
+    const size_t cap = (size_t)kMaxSplit * c->F_max * c->T * c->H * (c->D + 2) * sizeof(float);
+    return attend_impl(c, layer, out, out_dtype, stream, c->part_o, cap);
+}
+
+rtv_status rtv_attend_static_scratch(rtv_cache* c, int layer, void* out, int out_dtype, void* stream)
+{
+    if (!c) return RTV_ERR_INVALID_ARG;
+    if (!same_device(c)) return RTV_ERR_INVALID_ARG;
+    float* base = nullptr;
+    const rtv_status st = static_scratch_address(c->device, &base);
+    if (st != RTV_OK) return st;
+    return attend_impl(c, layer, out, out_dtype, stream, base, kStaticScratchFloats * sizeof(float));
 }
 
 rtv_status rtv_cache_advance(rtv_cache* c)

@@ -65,6 +65,7 @@ _SIGS = {
     "rtv_cache_destroy": (_S, [_P]),
     "rtv_cache_append": (_S, [_P, _S, _P, _P, _P, _S, _P]),
     "rtv_attend": (_S, [_P, _S, _P, _S, _P]),
+    "rtv_attend_static_scratch": (_S, [_P, _S, _P, _S, _P]),
     "rtv_cache_advance": (_S, [_P]),
     "rtv_cache_get_state": (_S, [_P, ctypes.POINTER(rtv_cache_state)]),
     "rtv_cache_device_buffer": (_S, [_P, ctypes.POINTER(_P), ctypes.POINTER(ctypes.c_size_t)]),
@@ -176,6 +177,14 @@ class Cache:
         if out.dtype not in (torch.bfloat16, torch.float32):
             return RTV_ERR_INVALID_ARG
         return lib.rtv_attend(self.handle, layer, _ptr(out), dt, _stream_ptr(stream))
+
+    def attend_static_scratch(self, layer: int, out, stream=None) -> int:
+        """rtv_attend with the split partials in the library's fixed device array."""
+        import torch
+        dt = RTV_OUT_BF16 if out.dtype == torch.bfloat16 else RTV_OUT_F32
+        if out.dtype not in (torch.bfloat16, torch.float32):
+            return RTV_ERR_INVALID_ARG
+        return lib.rtv_attend_static_scratch(self.handle, layer, _ptr(out), dt, _stream_ptr(stream))
 
     def advance(self) -> int:
         return lib.rtv_cache_advance(self.handle)
