@@ -11,6 +11,12 @@ rtv_attend (FP8 tcgen05 attention over the ring), then rtv_cache_advance
 above L2 too.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+    python bench.py --workload seq48 [--steps K] [--warmup W]
+
+--workload seq48 times the 48-layer step at the same shape instead (every
+layer appended and attended, then one advance; the ring full), reporting ms
+per step and the spread of the per-layer times; it prints a line of its own
+and is not the headline metric.
 
 N > 1 runs N independent replicas (one per GPU, launched by torchrun); the
 path has no data exchange, the process group only carries the barrier and
@@ -219,6 +225,62 @@ def us_per_layer_step(elapsed_ms: float, steps: int, world: int) -> float:
     return elapsed_ms * 1e3 / (steps * world)
 
 
+def run_seq48(args):
+    """48 layers x (append + attend), then advance, per step; one GPU."""
+    import torch
+    from kv_cache_serving_append_b200 import configs, rtv, synth
+    cfg = configs.get(4)
+    wl = workload(cfg)
+    L = cfg["n_layers"]
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    cache = rtv.Cache(cfg)
+    sets = [synth.chunk(4, cfg, 0, 100 + i, 1, device=dev) for i in range(N_INPUT_SETS)]
+    out = torch.empty((wl["T"], wl["H"], wl["D"]), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(i, ev=None):
+        for layer in range(L):
+            q, k, v = sets[(i * L + layer) % N_INPUT_SETS]
+            if ev is not None:
+                ev[layer][0].record(stream)
+            if cache.append(layer, q, k, v, 1, stream) or cache.attend(layer, out, stream):
+                raise RuntimeError("append/attend failed")
+            if ev is not None:
+                ev[layer][1].record(stream)
+        if cache.advance():
+            raise RuntimeError("advance failed")
+
+    for i in range(cfg["window_frames"] + 1 + args.warmup):   # fill the ring, warm up
+        step(i)
+    torch.cuda.synchronize()
+    evs = [[[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(L)]
+           for _ in range(args.steps)]
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for i in range(args.steps):
+        step(i, evs[i])
+    t1.record(stream)
+    torch.cuda.synchronize()
+    if cache.poll_error():
+        raise RuntimeError("kernel error in the timed region")
+    ms = t0.elapsed_time(t1) / args.steps
+    per_layer = [statistics.mean(evs[i][l][0].elapsed_time(evs[i][l][1]) for i in range(args.steps)) * 1e3
+                 for l in range(L)]
+    line = {"metric": "ms per 48-layer step (append+attn per layer, then advance) at full shape",
+            "value": ms, "unit": "ms/step", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+            "higher_is_better": False, "data": "synthetic",
+            "config": {"workload": "48 layers x (append + attend), 40 heads x D128, 2992 tokens/frame, "
+                                   "W=8, ring full", "cache_bytes": cache.nbytes},
+            "per_layer_us": {"mean": statistics.mean(per_layer), "stdev": statistics.pstdev(per_layer),
+                             "min": min(per_layer), "max": max(per_layer)},
+            "attend_key_splits": cache.state().last_attend_splits}
+    cache.close()
+    print(json.dumps(line))
+    return 0
+
+
 def run_reference(args):
     """--impl reference: the CPU oracle as it stands, on the host cores."""
     rank = int(os.environ.get("RANK", "0"))
@@ -272,9 +334,12 @@ def main():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--workload", default="layer", choices=["layer", "seq48"])
     args = ap.parse_args()
     if args.impl == "reference":
         return run_reference(args)
+    if args.workload == "seq48":
+        return run_seq48(args)
 
     import torch
     import torch.distributed as dist
