@@ -239,6 +239,18 @@ rtv_status rtv_cache_export(const rtv_cache* cache, int layer, int slot, void* c
 rtv_status rtv_poll_error(rtv_cache* cache);
 
 /*
+ * The key-range split rtv_attend chooses (host arithmetic only; no device
+ * needed).  n_units = ceil(n_frames*T / 256) * n_heads CTAs of one key range
+ * each, n_kv_tiles = key frames * ceil(T / 64), sm_count = the device's SMs.
+ * Out: n_split in 1..4 and tiles_per_split (the last split may hold fewer,
+ * none is empty).  The plan minimises ceil(n_units*s / sm_count) / s plus 3%
+ * per extra split, with at least 8 KV tiles per split.
+ * Errors: RTV_ERR_INVALID_ARG (a count < 1 or a NULL output).
+ */
+rtv_status rtv_split_plan(int n_units, int n_kv_tiles, int sm_count, int* n_split,
+                          int* tiles_per_split);
+
+/*
  * rtv_attend for callers that cannot allocate device memory: the same
  * kernels and results (bit for bit), but the key-range split partials go to a
  * fixed 16 MiB device array compiled into the library (file-scope

@@ -395,6 +395,29 @@ rtv_status rtv_cache_append(rtv_cache* c, int layer, const void* q, const void* 
     return RTV_OK;
 }
 
+rtv_status rtv_split_plan(int n_units, int n_kv_tiles, int sm_count, int* n_split, int* tiles_per_split)
+{
+    if (n_units < 1 || n_kv_tiles < 1 || sm_count < 1 || !n_split || !tiles_per_split)
+        return RTV_ERR_INVALID_ARG;
+    // One CTA per unit alone gives ceil(units / SMs) waves of equal CTAs;
+    // splitting every unit's key range s ways fills the last wave better at
+    // the price of a merge pass.  Pick s with the least ceil(units * s / SMs)
+    // / s, charging 3% of a full-range CTA per extra split (pipeline fill and
+    // drain, partial write and merge), and keep at least 8 KV tiles per split.
+    int best_s = 1;
+    double best_cost = 1e30;
+    for (int s = 1; s <= kMaxSplit; ++s) {
+        if (s > 1 && n_kv_tiles / s < 8) break;
+        const long long waves = ((long long)n_units * s + sm_count - 1) / sm_count;
+        const double cost = (double)waves / s + 0.03 * (s - 1);
+        if (cost < best_cost - 1e-9) { best_cost = cost; best_s = s; }
+    }
+    const int tps = (n_kv_tiles + best_s - 1) / best_s;
+    *tiles_per_split = tps;
+    *n_split = (n_kv_tiles + tps - 1) / tps;   // no empty split
+    return RTV_OK;
+}
+
 namespace {
 
 // Attention launch shared by rtv_attend and rtv_attend_static_scratch.  The
@@ -426,24 +449,9 @@ rtv_status attend_impl(rtv_cache* c, int layer, void* out, int out_dtype, void* 
     for (int s : c->visible_slots) p.slot[nk++] = s;
     for (int f = 0; f < n; ++f) p.slot[nk++] = staged_slot(c, f);
     p.n_frames_keys = nk;
-    // Key-range splits: one CTA per (head, 256 query rows) alone gives
-    // ceil(units / SMs) waves of equal CTAs; splitting every unit's key range
-    // s ways fills the last wave better at the price of a merge pass.  Pick s
-    // with the least ceil(units * s / SMs) / s, charging 3% of a full-range
-    // CTA per extra split (pipeline fill and drain, partial write and merge),
-    // and keep at least 8 KV tiles per split.
     const int units = ((p.M + 2 * kAttendRows - 1) / (2 * kAttendRows)) * p.H;
-    const int n_all = nk * p.tiles_per_frame;
-    int best_s = 1;
-    double best_cost = 1e30;
-    for (int s = 1; s <= kMaxSplit; ++s) {
-        if (s > 1 && n_all / s < 8) break;
-        const long long waves = ((long long)units * s + c->sm_count - 1) / c->sm_count;
-        const double cost = (double)waves / s + 0.03 * (s - 1);
-        if (cost < best_cost - 1e-9) { best_cost = cost; best_s = s; }
-    }
-    p.tiles_per_split = (n_all + best_s - 1) / best_s;
-    p.n_split = (n_all + p.tiles_per_split - 1) / p.tiles_per_split;   // no empty split
+    if (rtv_split_plan(units, nk * p.tiles_per_frame, c->sm_count, &p.n_split, &p.tiles_per_split) != RTV_OK)
+        return RTV_ERR_INVALID_ARG;
     const size_t part_rows = (size_t)p.n_split * p.M * p.H;
     if (p.n_split > 1 && part_rows * (p.D + 2) * sizeof(float) > capacity_bytes) return RTV_ERR_UNSUPPORTED;
     p.part_o = part_base;

@@ -66,6 +66,7 @@ _SIGS = {
     "rtv_cache_append": (_S, [_P, _S, _P, _P, _P, _S, _P]),
     "rtv_attend": (_S, [_P, _S, _P, _S, _P]),
     "rtv_attend_static_scratch": (_S, [_P, _S, _P, _S, _P]),
+    "rtv_split_plan": (_S, [_S, _S, _S, ctypes.POINTER(_S), ctypes.POINTER(_S)]),
     "rtv_cache_advance": (_S, [_P]),
     "rtv_cache_get_state": (_S, [_P, ctypes.POINTER(rtv_cache_state)]),
     "rtv_cache_device_buffer": (_S, [_P, ctypes.POINTER(_P), ctypes.POINTER(ctypes.c_size_t)]),
@@ -110,6 +111,13 @@ def make_config(cfg: dict) -> rtv_cache_config:
                             cfg["grid_w"], cfg["max_frames_per_chunk"], cfg["window_frames"],
                             cfg["pinned_frames"], cfg["rope_t"], cfg["rope_h"], cfg["rope_w"],
                             float(cfg.get("rope_base", 10000.0)))
+
+
+def split_plan(n_units: int, n_kv_tiles: int, sm_count: int):
+    """(n_split, tiles_per_split) that rtv_attend uses for this problem."""
+    a, b = _S(), _S()
+    check(lib.rtv_split_plan(n_units, n_kv_tiles, sm_count, ctypes.byref(a), ctypes.byref(b)), "rtv_split_plan")
+    return a.value, b.value
 
 
 def required_bytes(cfg: dict) -> int:

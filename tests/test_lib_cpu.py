@@ -116,3 +116,30 @@ def test_injected_allocation_failure_returns_oom():
                          cwd=ROOT, timeout=300)
     assert out.returncode == 0, out.stderr
     assert out.stdout.split() == ["2", "None"]
+
+
+def test_split_plan_choices_and_invariants(rtv):
+    """The key-range split rtv_attend uses (host arithmetic, no device)."""
+    # full-shape layer, ring full: 12 row blocks x 40 heads, 9 frames x 47 tiles, 148 SMs:
+    # 480 CTAs = 3.24 waves unsplit; 4 splits of <= 106 tiles -> 13 waves of quarter CTAs
+    assert rtv.split_plan(480, 9 * 47, 148) == (4, 106)
+    # the same layer's first step (one frame of keys): still 4 splits, of 12 tiles (last 11)
+    assert rtv.split_plan(480, 47, 148) == (4, 12)
+    # two frames per chunk, W=16 + pinned: 24 x 40 units, 19 x 47 tiles -> 2 splits
+    assert rtv.split_plan(960, 19 * 47, 148) == (2, 447)
+    # 704-token frames, 8 heads, 7 frames of 11 tiles: 24 units fill a fraction of the GPU
+    assert rtv.split_plan(24, 77, 148) == (4, 20)
+    # too few tiles to split (fewer than 8 per split)
+    assert rtv.split_plan(2, 5, 148) == (1, 5)
+    assert rtv.split_plan(480, 15, 148) == (1, 15)
+    for units in (1, 7, 148, 149, 296, 480, 960, 1500):
+        for tiles in (1, 8, 15, 16, 17, 47, 423, 1000):
+            s, tps = rtv.split_plan(units, tiles, 148)
+            assert 1 <= s <= 4
+            assert (s - 1) * tps < tiles <= s * tps          # every split non-empty, all tiles covered
+            if s > 1:
+                assert tps >= 8
+    n, t = ctypes.c_int(), ctypes.c_int()
+    for bad in ((0, 1, 148), (1, 0, 148), (1, 1, 0)):
+        assert rtv.lib.rtv_split_plan(*bad, ctypes.byref(n), ctypes.byref(t)) == 1
+    assert rtv.lib.rtv_split_plan(1, 1, 1, None, ctypes.byref(t)) == 1
