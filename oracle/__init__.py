@@ -201,4 +201,42 @@ def attend(qc, sq, kc, sk, vc, sv, rows=None, want_psum: bool = False):
     return (out, psum) if want_psum else out
 
 
+def attend_matmul(qc, sq, kc, sk, vc, sv, rows=None, block_rows: int = 512):
+    """The same fp64 attention as :func:`attend`, written with library
+    matrix products (PyTorch CPU, float64) as its steps:
+
+        Q^ = decode(qc) * sq,  K^ = decode(kc) * sk,  V^ = decode(vc) * sv
+        S  = (Q^ K^T) * (1 / sqrt(D))
+        P  = exp(S - rowmax(S))
+        O  = (P V^) / rowsum(P)
+
+    Every number is the definition's; only the order in which the products
+    of one dot product are added differs from the C loops (fp64 rounding,
+    about 1e-15 relative).  It exists so that the full output of a
+    full-shape call (millions of query-key pairs per head) can be computed
+    in seconds; the tests pin it to :func:`attend` and to PyTorch's float64
+    scaled_dot_product_attention.  Same arguments and output as
+    :func:`attend` (without ``want_psum``).
+    """
+    import torch
+    qc = np.ascontiguousarray(qc, np.uint8)
+    H, M, D = qc.shape
+    NK = kc.shape[1]
+    assert kc.shape == (H, NK, D) and vc.shape == (H, NK, D)
+    lut = e4m3_decode(np.arange(256, dtype=np.uint8))
+    rows = np.arange(M, dtype=np.int64) if rows is None else np.asarray(rows, np.int64)
+    out = np.empty((rows.size, H, D), np.float64)
+    inv_sqrt_d = 1.0 / np.sqrt(float(D))
+    for h in range(H):
+        qd = torch.from_numpy(lut[qc[h][rows]] * np.asarray(sq[h], np.float64)[rows, None])
+        kd = torch.from_numpy(lut[kc[h]] * np.asarray(sk[h], np.float64)[:, None])
+        vd = torch.from_numpy(lut[vc[h]] * np.asarray(sv[h], np.float64)[:, None])
+        for r0 in range(0, rows.size, block_rows):
+            s = torch.mm(qd[r0:r0 + block_rows], kd.T).mul_(inv_sqrt_d)    # S
+            p = s.sub_(s.max(dim=1, keepdim=True).values).exp_()          # P (in place)
+            o = torch.mm(p, vd).div_(p.sum(dim=1, keepdim=True))         # O
+            out[r0:r0 + block_rows, h] = o.numpy()
+    return out
+
+
 from .ring import OracleRing, OracleCache  # noqa: E402,F401

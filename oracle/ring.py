@@ -153,12 +153,18 @@ class OracleCache:
         sv = np.concatenate([L["sv"][s] for s in slots], axis=1)
         return slots, kc, sk, vc, sv
 
-    def attend(self, layer: int, rows=None, want_psum=False):
-        from . import attend
+    def attend(self, layer: int, rows=None, want_psum=False, matmul=False):
+        """fp64 attention of the staged chunk over the key set; ``matmul``
+        selects the library-matmul form of the same definition (for
+        full-shape outputs)."""
+        from . import attend, attend_matmul
         L = self.layers[layer]
         if L["staged"] == 0:
             raise RuntimeError("layer has no staged frames")
         _, kc, sk, vc, sv = self.key_set(layer)
+        if matmul:
+            assert not want_psum
+            return attend_matmul(L["qc"], L["sq"], kc, sk, vc, sv, rows=rows)
         return attend(L["qc"], L["sq"], kc, sk, vc, sv, rows=rows, want_psum=want_psum)
 
     def advance(self):

@@ -162,3 +162,63 @@ def test_tiny_workload_matches_torch_sdpa_fp64():
         assert np.max(np.abs(out - ref)) <= 1e-12 * max(1.0, np.abs(ref).max())
         assert kc.shape[1] == (min(step, cfg["window_frames"]) + 1) * 64
         cache.advance()
+
+
+def test_matmul_form_agrees_with_the_loops():
+    """The library-matmul form of the attention gives the C loops' result to
+    fp64 rounding, on random codes with spread scales, all rows and a row
+    sample, and with a key count that is not a multiple of anything."""
+    rng = np.random.default_rng(4)
+    for H, M, NK, D in [(2, 37, 301, 64), (3, 129, 1000, 128)]:
+        qc, kc, vc = _rand_codes(rng, (H, M, D)), _rand_codes(rng, (H, NK, D)), _rand_codes(rng, (H, NK, D))
+        sq, sk, sv = [rng.uniform(1e-3, 2e-2, s).astype(np.float32) for s in [(H, M), (H, NK), (H, NK)]]
+        ref = oracle.attend(qc, sq, kc, sk, vc, sv)
+        got = oracle.attend_matmul(qc, sq, kc, sk, vc, sv, block_rows=50)
+        assert np.max(np.abs(got - ref)) <= 1e-12 * max(1.0, np.abs(ref).max())
+        rows = np.array([M - 1, 0, M // 2], np.int32)
+        sub = oracle.attend_matmul(qc, sq, kc, sk, vc, sv, rows=rows, block_rows=50)
+        assert np.max(np.abs(sub - got[rows])) <= 1e-12 * max(1.0, np.abs(ref).max())
+
+
+def test_matmul_form_invariants():
+    """Equal keys give the mean of V; a dominant key gives its value."""
+    rng = np.random.default_rng(5)
+    H, M, NK, D = 1, 4, 96, 64
+    qc = _rand_codes(rng, (H, M, D))
+    kc = np.repeat(_rand_codes(rng, (H, 1, D)), NK, axis=1)
+    vc = _rand_codes(rng, (H, NK, D))
+    sq = np.full((H, M), 0.01, np.float32)
+    sk = np.full((H, NK), 0.02, np.float32)
+    sv = rng.uniform(0.1, 1, (H, NK)).astype(np.float32)
+    vhat = oracle.e4m3_decode(vc) * sv[..., None].astype(np.float64)
+    out = oracle.attend_matmul(qc, sq, kc, sk, vc, sv)
+    assert np.allclose(out, vhat.mean(axis=1)[None], rtol=0, atol=1e-12 * np.abs(vhat).max())
+    qc = np.full((H, M, D), 0x38, np.uint8)
+    kc = np.zeros((H, NK, D), np.uint8)
+    kc[0, 17] = 0x38
+    out = oracle.attend_matmul(qc, np.ones((H, M), np.float32), kc, np.full((H, NK), 4.0, np.float32),
+                               vc, np.ones((H, NK), np.float32))
+    v17 = oracle.e4m3_decode(vc[0, 17])
+    assert np.allclose(out[:, 0], v17[None], atol=np.abs(oracle.e4m3_decode(vc)).max() * NK * np.exp(-32) * 2)
+
+
+def test_matmul_form_matches_torch_sdpa_fp64_on_the_small_workload():
+    """Config 2 (8 heads, 704 tokens, outlier channels) after the ring has
+    wrapped, against PyTorch's float64 scaled_dot_product_attention on the
+    oracle's dequantised tensors."""
+    cfg = configs.get(2)
+    cache = oracle.OracleCache(cfg, layers=[0])
+    for step in range(cfg["window_frames"] + 2):
+        q, k, v = synth.chunk(2, cfg, 0, step, 1)
+        cache.append(0, synth.bf16_bits(q), synth.bf16_bits(k), synth.bf16_bits(v), 1)
+        if step < cfg["window_frames"] + 1:
+            cache.advance()
+    L = cache.layers[0]
+    _, kc, sk, vc, sv = cache.key_set(0)
+    out = cache.attend(0, matmul=True)
+    qh = torch.from_numpy(oracle.e4m3_decode(L["qc"]) * L["sq"][..., None].astype(np.float64))
+    kh = torch.from_numpy(oracle.e4m3_decode(kc) * sk[..., None].astype(np.float64))
+    vh = torch.from_numpy(oracle.e4m3_decode(vc) * sv[..., None].astype(np.float64))
+    ref = torch.nn.functional.scaled_dot_product_attention(qh[None], kh[None], vh[None])[0]
+    ref = ref.permute(1, 0, 2).numpy()
+    assert np.max(np.abs(out - ref)) <= 1e-12 * max(1.0, np.abs(ref).max())
