@@ -177,13 +177,19 @@ rtv_status rtv_cache_destroy(rtv_cache* cache);
  * 3D RoPE to Q and K, computes each (token, head) row's amax and scale, and
  * writes E4M3 codes and fp32 scales -- K and V into the ring slots of the
  * staged frames, Q into the layer's Q workspace.
+ * Source: aidose.in, "Runway explains how it serves a 57B video model in real
+ * time", third paragraph (rotary embedding and FP8 quantisation are applied
+ * once, when a frame is written into the cache); pttl.gr, section "Από οκτώ
+ * H100 σε τέσσερις", second paragraph (the same write-time transformation).
  *   q, k, v   bf16 [n_frames * T][n_heads][head_dim], row-major (the hidden
  *             dimension n_heads*head_dim contiguous), 16-byte aligned, not
- *             modified; read once.
+ *             modified; read once.  Owned by the caller; only read while the
+ *             launched kernel runs (stream-ordered).
  *   n_frames  1..max_frames_per_chunk (exactly 1 for the pinned chunk).
  * Absolute frame index of staged frame f = frames_committed + f.  Appending
  * again to the same layer before rtv_cache_advance overwrites its staged
- * frames (several denoising passes per chunk).
+ * frames (several denoising passes per chunk).  The library cannot check the
+ * sizes of q/k/v: the caller passes n_frames*T*n_heads*head_dim elements each.
  * Errors: RTV_ERR_INVALID_ARG (layer, n_frames, NULL or misaligned pointer),
  * RTV_ERR_STATE (layers staged with different frame counts), RTV_ERR_CUDA.
  */
@@ -192,7 +198,12 @@ rtv_status rtv_cache_append(rtv_cache* cache, int layer, const void* q, const vo
 
 /*
  * Attention of the layer's staged chunk over its key set (pinned frame,
- * window oldest to newest, staged frames), written to
+ * window oldest to newest, staged frames).
+ * Source: aidose.in, "Runway explains how it serves a 57B video model in real
+ * time", third paragraph (attention runs over the cache whose frames were
+ * rotated and quantised at write time); pttl.gr, section "Από οκτώ H100 σε
+ * τέσσερις", second paragraph (240 attention calls per diffusion step).
+ * The result is written to
  *   out  [n_frames * T][n_heads][head_dim], fp32 (RTV_OUT_F32) or bf16
  *        (RTV_OUT_BF16), row-major, 16-byte aligned.
  * One kernel: TMA loads of Q/K/V codes and scales by (slot, head, token
@@ -213,7 +224,10 @@ rtv_status rtv_attend(rtv_cache* cache, int layer, void* out, int out_dtype, voi
 /*
  * Commit the staged frames of every layer (host bookkeeping only; launches
  * nothing and copies nothing).  Requires all layers staged with the same
- * frame count.  Errors: RTV_ERR_STATE.
+ * frame count.  Source: aidose.in, "Runway explains how it serves a 57B video
+ * model in real time", third paragraph (the cache is a ring buffer that moves
+ * forward without copying); pttl.gr, section "Από οκτώ H100 σε τέσσερις",
+ * second paragraph (circular buffer).  Errors: RTV_ERR_STATE.
  */
 rtv_status rtv_cache_advance(rtv_cache* cache);
 
@@ -224,12 +238,19 @@ rtv_status rtv_cache_get_state(const rtv_cache* cache, rtv_cache_state* out);
 rtv_status rtv_cache_device_buffer(const rtv_cache* cache, void** ptr, size_t* bytes);
 
 /*
- * Copy one slot of one layer to HOST buffers (test and debug use; waits for
- * the stream).  codes_k/codes_v: [n_heads][T][head_dim] bytes; sk/sv:
- * [n_heads][T] floats.  Any pointer may be NULL to skip that tensor.
+ * Copy one slot of one layer, and the layer's Q workspace, to HOST buffers
+ * (test and debug use; waits for the stream).
+ *   codes_k, codes_v  [n_heads][T][head_dim] bytes of the slot
+ *   sk, sv            [n_heads][T] floats of the slot
+ *   q_codes           [n_heads][max_frames_per_chunk * T][head_dim] bytes
+ *   sq                [n_heads][max_frames_per_chunk * T] floats
+ * (the Q workspace rows of the staged frames come first).  Any pointer may be
+ * NULL to skip that tensor.  Errors: RTV_ERR_INVALID_ARG (layer, slot),
+ * RTV_ERR_CUDA.
  */
 rtv_status rtv_cache_export(const rtv_cache* cache, int layer, int slot, void* codes_k,
-                            void* codes_v, float* sk, float* sv, void* stream);
+                            void* codes_v, float* sk, float* sv, void* q_codes, float* sq,
+                            void* stream);
 
 /*
  * Read (and clear) the device error word.  Synchronises the device; the only
@@ -254,16 +275,21 @@ rtv_status rtv_split_plan(int n_units, int n_kv_tiles, int sm_count, int* n_spli
  * rtv_attend for callers that cannot allocate device memory: the same
  * kernels and results (bit for bit), but the key-range split partials go to a
  * fixed 16 MiB device array compiled into the library (file-scope
- * __device__, its address looked up once per device) instead of the cache
- * buffer's split section.  The call allocates nothing (no cudaMalloc/
- * cudaFree, no allocating library routine).  Nothing in the array needs to
- * start at zero: the merge reads only partials the same call wrote.  The array
- * is shared by every cache and stream on the device: calls that overlap in
- * time (other streams, other host threads) race.  A call whose split plan
- * needs more than 16 MiB of partials (n_split x n_frames*T x n_heads x
- * (head_dim + 2) fp32) is rejected with RTV_ERR_UNSUPPORTED before anything
- * is launched; an unsplit call needs none.  The method's sources describe no
- * counterpart of this entry point: it is a deployment convenience.
+ * __device__) instead of the cache buffer's split section.  The call
+ * allocates nothing (no cudaMalloc/cudaFree, no allocating library routine).
+ * Device footprint: every device on which a cache is created holds the
+ * 16 MiB array until the process exits -- rtv_cache_create looks up its
+ * address (once per device, with that device current), which makes the
+ * CUDA runtime load the module that holds it; if that lookup failed there,
+ * the first call of this entry point retries it.  Nothing in the array needs
+ * to start at zero: the merge reads only partials the same call wrote.  The
+ * array is shared by every cache and stream on the device: calls that
+ * overlap in time (other streams, other host threads) race.  A call whose
+ * split plan needs more than 16 MiB of partials (n_split x n_frames*T x
+ * n_heads x (head_dim + 2) fp32) is rejected with RTV_ERR_UNSUPPORTED before
+ * anything is launched; an unsplit call needs none.  The method's sources
+ * describe no counterpart of this entry point: it is a deployment
+ * convenience.
  * Errors: as rtv_attend, plus RTV_ERR_UNSUPPORTED (partials over 16 MiB) and
  * RTV_ERR_CUDA (symbol lookup failed).
  */

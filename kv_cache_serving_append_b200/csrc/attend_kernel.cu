@@ -54,6 +54,8 @@
 #include <cuda_fp16.h>
 #include <cuda_fp8.h>
 
+#include <mutex>
+
 #include "rtv_internal.h"
 #include "sm100.cuh"
 
@@ -628,19 +630,33 @@ __global__ void __launch_bounds__(256) combine_kernel(const AttendParams p)
     }
 }
 
+// Raise the kernel's dynamic shared-memory limit once per device (the
+// attribute is per device and per function); guarded for concurrent callers.
+template <int D>
+cudaError_t configure_once(int dev, size_t smem)
+{
+    static std::mutex mu;
+    static bool done[kMaxDevices] = {};
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!done[dev]) {
+        cudaError_t e = cudaFuncSetAttribute(attend_kernel<D>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        done[dev] = true;
+    }
+    return cudaSuccess;
+}
+
 template <int D>
 cudaError_t launch(const AttendParams& p, const CUtensorMap* maps, cudaStream_t stream)
 {
     const size_t smem = sizeof(Smem<D>) + 1024;
     int dev = 0;
-    cudaGetDevice(&dev);
-    static unsigned configured = 0;   // bit per device
-    if (dev < 32 && !(configured & (1u << dev))) {
-        cudaError_t e = cudaFuncSetAttribute(attend_kernel<D>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-        configured |= 1u << dev;
-    }
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    e = configure_once<D>(dev, smem);
+    if (e != cudaSuccess) return e;
     dim3 grid((p.M + kQT * kBM - 1) / (kQT * kBM), p.H, p.n_split);
     attend_kernel<D><<<grid, kThreads, smem, stream>>>(p, maps[0], maps[1], maps[2], maps[3], maps[4]);
     if (p.n_split > 1) {

@@ -218,6 +218,30 @@ int staged_slot(const rtv_cache* c, int f)
     return c->P0 + (int)((c->G + f) % c->C);
 }
 
+// Split partials of rtv_attend_static_scratch: a fixed device array (16 MiB),
+// shared by every cache and stream of the device.
+constexpr size_t kStaticScratchFloats = (size_t)4 << 20;
+__device__ __align__(256) float g_static_scratch[kStaticScratchFloats];
+
+// Address of g_static_scratch on the current device, looked up once per device.
+rtv_status static_scratch_address(int device, float** out)
+{
+    static std::mutex mu;
+    static void* addr[kMaxDevices] = {};
+    if (device < 0 || device >= kMaxDevices) return RTV_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!addr[device]) {
+        void* a = nullptr;
+        if (cudaGetSymbolAddress(&a, g_static_scratch) != cudaSuccess || !a) {
+            cudaGetLastError();
+            return RTV_ERR_CUDA;
+        }
+        addr[device] = a;
+    }
+    *out = static_cast<float*>(addr[device]);
+    return RTV_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -320,6 +344,15 @@ rtv_status rtv_cache_create(const rtv_cache_config* cfg, void* device_buf, size_
     if (ok && !wt.empty())
         ok = cudaMemcpy(c->w_table, wt.data(), wt.size() * 4, cudaMemcpyHostToDevice) == cudaSuccess;
     if (ok) ok = cudaDeviceSynchronize() == cudaSuccess;
+    if (ok) {
+        // Resolve the allocation-free entry point's device array now, so the
+        // module that holds it is loaded at set-up (under lazy module loading
+        // its 16 MiB are reserved here, not by a later attention call).  A
+        // failure is not fatal to the cache: rtv_attend_static_scratch then
+        // retries and reports it.
+        float* scratch = nullptr;
+        if (static_scratch_address(c->device, &scratch) != RTV_OK) cudaGetLastError();
+    }
     if (ok && !build_maps(c)) {
         if (c->owns) cudaFree(c->buf);
         delete c;
@@ -466,30 +499,6 @@ rtv_status attend_impl(rtv_cache* c, int layer, void* out, int out_dtype, void* 
     return RTV_OK;
 }
 
-// Split partials of rtv_attend_static_scratch: a fixed device array (16 MiB),
-// shared by every cache and stream of the device.
-constexpr size_t kStaticScratchFloats = (size_t)4 << 20;
-__device__ __align__(256) float g_static_scratch[kStaticScratchFloats];
-
-// Address of g_static_scratch on the current device, looked up once per device.
-rtv_status static_scratch_address(int device, float** out)
-{
-    static std::mutex mu;
-    static void* addr[64] = {};
-    if (device < 0 || device >= 64) return RTV_ERR_UNSUPPORTED;
-    std::lock_guard<std::mutex> lock(mu);
-    if (!addr[device]) {
-        void* a = nullptr;
-        if (cudaGetSymbolAddress(&a, g_static_scratch) != cudaSuccess || !a) {
-            cudaGetLastError();
-            return RTV_ERR_CUDA;
-        }
-        addr[device] = a;
-    }
-    *out = static_cast<float*>(addr[device]);
-    return RTV_OK;
-}
-
 }  // namespace
 
 rtv_status rtv_attend(rtv_cache* c, int layer, void* out, int out_dtype, void* stream)
@@ -577,7 +586,7 @@ rtv_status rtv_cache_device_buffer(const rtv_cache* c, void** ptr, size_t* bytes
 }
 
 rtv_status rtv_cache_export(const rtv_cache* c, int layer, int slot, void* codes_k, void* codes_v,
-                            float* sk, float* sv, void* stream)
+                            float* sk, float* sv, void* q_codes, float* sq, void* stream)
 {
     if (!c || layer < 0 || layer >= c->cfg.n_layers || slot < 0 || slot >= c->S)
         return RTV_ERR_INVALID_ARG;
@@ -591,7 +600,11 @@ rtv_status rtv_cache_export(const rtv_cache* c, int layer, int slot, void* codes
     const size_t sbase = (size_t)slot * c->H * pitch;
     if (sk) ok &= cudaMemcpy2DAsync(sk, (size_t)c->T * 4, c->buf + L.k_scales + sbase, pitch, (size_t)c->T * 4, c->H, cudaMemcpyDeviceToHost, s) == cudaSuccess;
     if (sv) ok &= cudaMemcpy2DAsync(sv, (size_t)c->T * 4, c->buf + L.v_scales + sbase, pitch, (size_t)c->T * 4, c->H, cudaMemcpyDeviceToHost, s) == cudaSuccess;
+    const size_t q_rows = (size_t)c->F_max * c->T;
+    if (q_codes) ok &= cudaMemcpyAsync(q_codes, c->buf + L.q_codes, (size_t)c->H * q_rows * c->D, cudaMemcpyDeviceToHost, s) == cudaSuccess;
+    if (sq) ok &= cudaMemcpy2DAsync(sq, q_rows * 4, c->buf + L.q_scales, (size_t)L.q_scale_pitch * 4, q_rows * 4, c->H, cudaMemcpyDeviceToHost, s) == cudaSuccess;
     if (ok) ok = cudaStreamSynchronize(s) == cudaSuccess;
+    if (!ok) cudaGetLastError();
     return ok ? RTV_OK : RTV_ERR_CUDA;
 }
 

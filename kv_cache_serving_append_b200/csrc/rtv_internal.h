@@ -20,6 +20,7 @@ constexpr int kMaxRopeHalf = 32;   // rope_t / 2 <= 32 (frame-axis table travels
 constexpr int kAttendRows = 128;
 constexpr int kAttendKeys = 64;
 constexpr int kMaxSplit = 4;       // key-range splits of one attention call
+constexpr int kMaxDevices = 64;    // per-device one-time set-up tables
 
 // Device error word bits.
 constexpr uint32_t kErrTimeout = 1u;

@@ -70,7 +70,7 @@ _SIGS = {
     "rtv_cache_advance": (_S, [_P]),
     "rtv_cache_get_state": (_S, [_P, ctypes.POINTER(rtv_cache_state)]),
     "rtv_cache_device_buffer": (_S, [_P, ctypes.POINTER(_P), ctypes.POINTER(ctypes.c_size_t)]),
-    "rtv_cache_export": (_S, [_P, _S, _S, _P, _P, _P, _P, _P]),
+    "rtv_cache_export": (_S, [_P, _S, _S, _P, _P, _P, _P, _P, _P, _P]),
     "rtv_poll_error": (_S, [_P]),
     "rtv_debug_set_wait_fault": (_S, [_P, _S, ctypes.c_longlong]),
 }
@@ -153,6 +153,8 @@ class Cache:
         import torch
         self.cfg = dict(cfg)
         self.device = torch.device(device or "cuda")
+        if self.device.index is None:
+            self.device = torch.device("cuda", torch.cuda.current_device())
         self.nbytes = required_bytes(cfg)
         self.buffer = torch.empty(self.nbytes, dtype=torch.uint8, device=self.device)
         self._c = make_config(cfg)
@@ -162,6 +164,7 @@ class Cache:
                                        ctypes.byref(h)), "rtv_cache_create")
         self.handle = h
         self.T = cfg["grid_h"] * cfg["grid_w"]
+        self._staged = {}          # layer -> frames staged since the last advance
 
     def close(self):
         if self.handle:
@@ -174,34 +177,84 @@ class Cache:
         except Exception:
             pass
 
+    # -- argument checks (the C ABI sees bare pointers and cannot check sizes)
+    def tensor_status(self, t, numel: int, dtypes) -> int:
+        """RTV_OK if ``t`` is a contiguous tensor of one of ``dtypes`` with
+        ``numel`` elements on this cache's device, else RTV_ERR_INVALID_ARG.
+        A tensor that fails here never reaches the library: a short, strided
+        or foreign-device buffer would make a kernel read or write outside it."""
+        try:
+            ok = (t.dtype in dtypes and t.is_contiguous() and t.device == self.device
+                  and t.numel() == numel)
+        except AttributeError:
+            ok = False
+        return RTV_OK if ok else RTV_ERR_INVALID_ARG
+
+    def _rows(self, n_frames: int) -> int:
+        return n_frames * self.T * self.cfg["n_heads"] * self.cfg["head_dim"]
+
     # -- the hot path ----------------------------------------------------
     def append(self, layer: int, q, k, v, n_frames: int, stream=None) -> int:
-        return lib.rtv_cache_append(self.handle, layer, _ptr(q), _ptr(k), _ptr(v), n_frames,
-                                    _stream_ptr(stream))
+        import torch
+        if not isinstance(n_frames, int) or not 1 <= n_frames <= self.cfg["max_frames_per_chunk"]:
+            return RTV_ERR_INVALID_ARG
+        for t in (q, k, v):
+            st = self.tensor_status(t, self._rows(n_frames), (torch.bfloat16,))
+            if st != RTV_OK:
+                return st
+        st = lib.rtv_cache_append(self.handle, layer, _ptr(q), _ptr(k), _ptr(v), n_frames,
+                                  _stream_ptr(stream))
+        if st == RTV_OK:
+            self._staged[layer] = n_frames
+        return st
+
+    def _out_status(self, layer: int, out) -> tuple[int, int]:
+        import torch
+        n = self._staged.get(layer, 0)
+        if n == 0:
+            return RTV_OK, RTV_OUT_F32      # the library reports RTV_ERR_STATE (or a bad layer)
+        st = self.tensor_status(out, self._rows(n), (torch.float32, torch.bfloat16))
+        return st, (RTV_OUT_BF16 if getattr(out, "dtype", None) == torch.bfloat16 else RTV_OUT_F32)
 
     def attend(self, layer: int, out, stream=None) -> int:
-        import torch
-        dt = RTV_OUT_BF16 if out.dtype == torch.bfloat16 else RTV_OUT_F32
-        if out.dtype not in (torch.bfloat16, torch.float32):
-            return RTV_ERR_INVALID_ARG
+        st, dt = self._out_status(layer, out)
+        if st != RTV_OK:
+            return st
         return lib.rtv_attend(self.handle, layer, _ptr(out), dt, _stream_ptr(stream))
 
     def attend_static_scratch(self, layer: int, out, stream=None) -> int:
         """rtv_attend with the split partials in the library's fixed device array."""
-        import torch
-        dt = RTV_OUT_BF16 if out.dtype == torch.bfloat16 else RTV_OUT_F32
-        if out.dtype not in (torch.bfloat16, torch.float32):
-            return RTV_ERR_INVALID_ARG
+        st, dt = self._out_status(layer, out)
+        if st != RTV_OK:
+            return st
         return lib.rtv_attend_static_scratch(self.handle, layer, _ptr(out), dt, _stream_ptr(stream))
 
     def advance(self) -> int:
-        return lib.rtv_cache_advance(self.handle)
+        st = lib.rtv_cache_advance(self.handle)
+        if st == RTV_OK:
+            self._staged.clear()
+        return st
 
     # -- inspection ------------------------------------------------------
     def state(self) -> rtv_cache_state:
         st = rtv_cache_state()
         check(lib.rtv_cache_get_state(self.handle, ctypes.byref(st)), "rtv_cache_get_state")
         return st
+
+    def export(self, layer: int, slot: int, stream=None) -> dict:
+        """Host copies (numpy) of one slot's K/V codes and scales and of the
+        layer's Q workspace, through rtv_cache_export."""
+        import numpy as np
+        H, D, T = self.cfg["n_heads"], self.cfg["head_dim"], self.T
+        qr = self.cfg["max_frames_per_chunk"] * T
+        out = dict(k_codes=np.empty((H, T, D), np.uint8), v_codes=np.empty((H, T, D), np.uint8),
+                   k_scales=np.empty((H, T), np.float32), v_scales=np.empty((H, T), np.float32),
+                   q_codes=np.empty((H, qr, D), np.uint8), q_scales=np.empty((H, qr), np.float32))
+        a = lambda x: x.ctypes.data_as(ctypes.c_void_p)   # noqa: E731
+        check(lib.rtv_cache_export(self.handle, layer, slot, a(out["k_codes"]), a(out["v_codes"]),
+                                   a(out["k_scales"]), a(out["v_scales"]), a(out["q_codes"]),
+                                   a(out["q_scales"]), _stream_ptr(stream)), "rtv_cache_export")
+        return out
 
     def poll_error(self) -> int:
         return lib.rtv_poll_error(self.handle)

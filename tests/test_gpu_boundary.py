@@ -49,8 +49,10 @@ def test_pinned_chunk_is_one_frame(gpu):
     cfg.update(n_heads=2, grid_h=4, grid_w=8)
     c = rtv.Cache(cfg)
     q, k, v = (t.cuda() for t in synth.chunk(5, cfg, 0, -1, 2))
-    assert c.append(0, q, k, v, 2) == rtv.RTV_ERR_INVALID_ARG
-    assert c.append(0, q, k, v, 1) == rtv.RTV_OK
+    T = cfg["grid_h"] * cfg["grid_w"]
+    assert c.append(0, q, k, v, 2) == rtv.RTV_ERR_INVALID_ARG       # the library refuses 2 frames
+    assert c.append(0, q, k, v, 1) == rtv.RTV_ERR_INVALID_ARG       # the binding: 2 frames of rows
+    assert c.append(0, q[:T], k[:T], v[:T], 1) == rtv.RTV_OK
     assert c.advance() == rtv.RTV_OK
     st = c.state()
     assert st.pinned_committed == 1 and st.visible_slots[0] == 0 and st.frame_of_slot[0] == 0
@@ -110,25 +112,37 @@ def test_bounded_wait_times_out_and_context_survives(gpu):
 
 
 def test_library_allocated_buffer_and_export(gpu):
-    """rtv_cache_create with a NULL buffer (library cudaMalloc) and the
-    host export of one slot."""
+    """rtv_cache_create with a NULL buffer (library cudaMalloc), then the
+    host export (rtv_cache_export, through the C ABI) of the staged slot's K
+    and V codes and scales and of the Q workspace, each held to the parity
+    tolerance against the oracle: codes identical except one code step where
+    the oracle flags a rounding boundary, scales within 1e-6 relative."""
+    import oracle
     from kv_cache_serving_append_b200 import rtv
+    from parity import compare_codes, compare_scales
     cfg = configs.get(1)
+    H, D, T = cfg["n_heads"], cfg["head_dim"], 64
+    split = (cfg["rope_t"], cfg["rope_h"], cfg["rope_w"])
     c = rtv.make_config(cfg)
     h = ctypes.c_void_p()
     assert rtv.lib.rtv_cache_create(ctypes.byref(c), None, 0, ctypes.byref(h)) == 0
-    q, k, v = (t.cuda() for t in synth.chunk(1, cfg, 0, 0, 1))
     s = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
-    assert rtv.lib.rtv_cache_append(h, 0, ctypes.c_void_p(q.data_ptr()), ctypes.c_void_p(k.data_ptr()),
-                                    ctypes.c_void_p(v.data_ptr()), 1, s) == 0
-    kc = np.zeros((2, 64, 64), np.uint8)
-    sk = np.zeros((2, 64), np.float32)
-    assert rtv.lib.rtv_cache_export(h, 0, 0, kc.ctypes.data_as(ctypes.c_void_p), None,
-                                    sk.ctypes.data_as(ctypes.c_void_p), None, s) == 0
-    import oracle
-    oc, osk, near = oracle.append_tensor(synth.bf16_bits(k.cpu()), 64, 8, 0, True, (16, 24, 24))
-    assert np.array_equal(kc, oc) or np.all((kc == oc) | (near != 0))
-    assert np.array_equal(sk, osk)
+    a = lambda x: x.ctypes.data_as(ctypes.c_void_p)   # noqa: E731
+    for step in range(2):            # slot 0 at frame 0, then slot 1 at frame 1
+        q, k, v = (t.cuda() for t in synth.chunk(1, cfg, 0, step, 1))
+        assert rtv.lib.rtv_cache_append(h, 0, ctypes.c_void_p(q.data_ptr()), ctypes.c_void_p(k.data_ptr()),
+                                        ctypes.c_void_p(v.data_ptr()), 1, s) == 0
+        kc, vc = np.zeros((H, T, D), np.uint8), np.zeros((H, T, D), np.uint8)
+        sk, sv = np.zeros((H, T), np.float32), np.zeros((H, T), np.float32)
+        qc, sq = np.zeros((H, T, D), np.uint8), np.zeros((H, T), np.float32)
+        assert rtv.lib.rtv_cache_export(h, 0, step, a(kc), a(vc), a(sk), a(sv), a(qc), a(sq), s) == 0
+        for name, x, g, sg, rope in (("q", q, qc, sq, True), ("k", k, kc, sk, True), ("v", v, vc, sv, False)):
+            oc, osc, near = oracle.append_tensor(synth.bf16_bits(x.cpu()), T, cfg["grid_w"], step, rope, split)
+            r = compare_codes(g, oc, near)
+            assert r["bad"] == 0, (name, step, r)
+            assert compare_scales(sg, osc) == 0, (name, step)
+        assert rtv.lib.rtv_cache_advance(h) == 0
+    assert rtv.lib.rtv_cache_export(h, 0, 99, None, None, None, None, None, None, s) == rtv.RTV_ERR_INVALID_ARG
     ptr, nb = ctypes.c_void_p(), ctypes.c_size_t()
     assert rtv.lib.rtv_cache_device_buffer(h, ctypes.byref(ptr), ctypes.byref(nb)) == 0
     assert nb.value == rtv.required_bytes(cfg) and ptr.value

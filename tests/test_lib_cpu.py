@@ -143,3 +143,34 @@ def test_split_plan_choices_and_invariants(rtv):
     for bad in ((0, 1, 148), (1, 0, 148), (1, 1, 0)):
         assert rtv.lib.rtv_split_plan(*bad, ctypes.byref(n), ctypes.byref(t)) == 1
     assert rtv.lib.rtv_split_plan(1, 1, 1, None, ctypes.byref(t)) == 1
+
+
+def test_binding_rejects_bad_tensors_before_the_library(rtv):
+    """The binding checks dtype, contiguity, device and element count of every
+    tensor it would pass as a bare pointer, and answers RTV_ERR_INVALID_ARG
+    itself; here on CPU tensors against a cache object that has no library
+    handle (so nothing could be launched even if a check were missing)."""
+    import torch
+    from kv_cache_serving_append_b200 import configs
+    cfg = configs.get(1)
+    c = object.__new__(rtv.Cache)
+    c.cfg, c.T, c.handle, c._staged = cfg, 64, None, {}
+    c.device = torch.device("cpu")
+    n = 64 * cfg["n_heads"] * cfg["head_dim"]
+    good = torch.zeros((64, cfg["n_heads"], cfg["head_dim"]), dtype=torch.bfloat16)
+    assert c.tensor_status(good, n, (torch.bfloat16,)) == rtv.RTV_OK
+    assert c.tensor_status(good.float(), n, (torch.bfloat16,)) == rtv.RTV_ERR_INVALID_ARG   # dtype
+    assert c.tensor_status(good.transpose(0, 1), n, (torch.bfloat16,)) == rtv.RTV_ERR_INVALID_ARG  # strided
+    assert c.tensor_status(good[:32], n, (torch.bfloat16,)) == rtv.RTV_ERR_INVALID_ARG     # too short
+    assert c.tensor_status(None, n, (torch.bfloat16,)) == rtv.RTV_ERR_INVALID_ARG
+    c.device = torch.device("cuda", 0)
+    assert c.tensor_status(good, n, (torch.bfloat16,)) == rtv.RTV_ERR_INVALID_ARG          # device
+    # the hot-path calls answer from those checks
+    assert c.append(0, good, good, good, 1) == rtv.RTV_ERR_INVALID_ARG
+    assert c.append(0, good, good, good, 0) == rtv.RTV_ERR_INVALID_ARG
+    assert c.append(0, good, good, good, 2) == rtv.RTV_ERR_INVALID_ARG    # > max_frames_per_chunk
+    c._staged[0] = 1
+    out = torch.zeros((64, cfg["n_heads"], cfg["head_dim"]), dtype=torch.float32)
+    assert c.attend(0, out) == rtv.RTV_ERR_INVALID_ARG                     # CPU tensor
+    assert c.attend(0, out.half()) == rtv.RTV_ERR_INVALID_ARG
+    assert c.attend_static_scratch(0, out[:10]) == rtv.RTV_ERR_INVALID_ARG
