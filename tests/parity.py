@@ -61,11 +61,17 @@ def ring_state_matches(st, ring: oracle.OracleRing) -> None:
 
 
 def sample_rows(M: int, n: int, seed: int) -> np.ndarray:
-    """First and last rows (ragged tile tail) plus random ones."""
+    """About n query rows: the first and last rows and the ragged tail of the
+    last 128-row tile, plus random rows drawn from every 128-row tile alike."""
     rng = np.random.default_rng(seed)
     fixed = [0, 1, 127, 128, M - 1, M - 2, M - 48, (M // 128) * 128]
     fixed = [r for r in fixed if 0 <= r < M]
-    rest = rng.choice(M, size=min(M, max(0, n - len(fixed))), replace=False)
+    n_tiles = (M + 127) // 128
+    per_tile = max(1, -(-max(0, n - len(fixed)) // n_tiles))
+    rest = []
+    for t in range(n_tiles):
+        lo, hi = 128 * t, min(M, 128 * t + 128)
+        rest.extend(rng.choice(np.arange(lo, hi), size=min(per_tile, hi - lo), replace=False))
     return np.unique(np.concatenate([fixed, rest]).astype(np.int32))
 
 
@@ -128,7 +134,11 @@ class Runner:
         torch.cuda.synchronize()
         assert self.cache.poll_error() == 0
         g = out.float().cpu().numpy()
-        o = self.ora.attend(layer, rows=rows)
+        # large calls use the oracle's library-matmul form of the same
+        # definition (pinned to the C loops by the CPU tests)
+        nk = len(self.ora.ring.key_slots(n)) * self.T
+        big = (M if rows is None else len(rows)) * nk * self.H > 2e8
+        o = self.ora.attend(layer, rows=rows, matmul=big)
         if rows is not None:
             g = g[rows]
         assert np.isfinite(g).all()

@@ -1,11 +1,15 @@
 """GPU parity: the CUDA path through the C ABI against the oracle, on the
 seeded workloads, with the tolerances in tests/parity.py.
 
-Tiny and small workloads are compared element by element on every output at
-every step; the full-shape workloads compare every code and scale of every
-append and a sample of query rows of the attention output (first and last
-rows, the ragged tail of the last 128-row tile, and random rows), at steps
-that cover an empty, partly filled, full and wrapped ring.
+Every code and scale of every append is compared.  Attention outputs are
+compared element by element: at every step for the tiny and small
+workloads; for the full-shape layer and the long-window workload the whole
+output at steps after the ring has wrapped (the launch configuration the
+benchmark times, key range split included), and sampled query rows (first
+and last rows, the ragged tail of the last 128-row tile, random rows from
+every 128-row tile) at the steps that cover an empty, partly filled and
+just-full ring.  Chunks of 1 to 4 frames, with and without the pinned slot,
+run on small shapes at every step.
 """
 import numpy as np
 import pytest
@@ -18,8 +22,12 @@ pytestmark = pytest.mark.gpu
 
 
 def run_full_compare(cfg_id, steps=None, check_attn_steps=None, rows_per_step=None,
-                     out_dtype=torch.float32):
-    cfg = configs.get(cfg_id)
+                     full_steps=(), out_dtype=torch.float32, cfg=None):
+    """Drive a workload through the GPU cache and the oracle; compare every
+    append, and the attention output at ``check_attn_steps`` (all steps if
+    None): the whole output at ``full_steps`` or when ``rows_per_step`` is
+    None, else ``rows_per_step`` sampled rows."""
+    cfg = cfg or configs.get(cfg_id)
     R = Runner(cfg_id, cfg)
     worst = (0.0, 0.0)
     n_steps = cfg["steps"] if steps is None else steps
@@ -28,13 +36,15 @@ def run_full_compare(cfg_id, steps=None, check_attn_steps=None, rows_per_step=No
         for layer in range(cfg["n_layers"]):
             R.append(layer, step, F)
         for layer in range(cfg["n_layers"]):
-            if check_attn_steps is None or step in check_attn_steps:
+            if check_attn_steps is None or step in check_attn_steps or step in full_steps:
                 rows = None
-                if rows_per_step:
-                    rows = sample_rows(F * R.T, rows_per_step, 1000 * (step + 1) + layer)
+                if rows_per_step and step not in full_steps:
+                    rows = sample_rows(F * R.T, rows_per_step, 1000 * (step + 2) + layer)
                 g, o = R.attend(layer, rows=rows, out_dtype=out_dtype)
                 mx, rl = attn_errors(g, o)
                 worst = (max(worst[0], mx), max(worst[1], rl))
+                print(f"cfg {cfg_id} step {step} layer {layer} rows {'all' if rows is None else len(rows)}: "
+                      f"max-abs {mx:.4g} rel-L2 {rl:.4g} splits {R.cache.state().last_attend_splits}")
                 assert mx <= ATOL_MAX and rl <= REL_L2, (cfg_id, step, layer, mx, rl)
         R.advance()
     R.cache.close()
@@ -51,18 +61,82 @@ def test_small_every_step_full_output(gpu):
     print("config 2 worst max-abs %.3g rel-L2 %.3g" % worst)
 
 
-def test_full_shape_layer_sampled_rows(gpu):
+def test_full_shape_layer_full_output_after_wrap(gpu):
+    """Config 3: the whole output (2992 rows x 40 heads) at the first step
+    whose ring has wrapped and at the next, sampled rows before."""
     cfg = configs.get(3)
     W = cfg["window_frames"]
-    worst = run_full_compare(3, steps=W + 3, check_attn_steps={0, 1, W - 1, W, W + 2},
-                             rows_per_step=48)
+    worst = run_full_compare(3, steps=W + 4, check_attn_steps={0, 1, W - 1, W},
+                             rows_per_step=256, full_steps=(W + 2, W + 3))
     print("config 3 worst max-abs %.3g rel-L2 %.3g" % worst)
 
 
-def test_long_window_pinned_sampled_rows(gpu):
-    worst = run_full_compare(5, steps=None, check_attn_steps={-1, 0, 1, 7, 8, 9, 23},
-                             rows_per_step=40)
+def test_long_window_pinned_full_output_after_wrap(gpu):
+    """Config 5: the pinned chunk, the filling ring with 640 sampled rows (every
+    128-row tile), and the whole output (5984 rows x 40 heads) at the last
+    step, long after the ring wrapped."""
+    worst = run_full_compare(5, steps=None, check_attn_steps={-1, 0, 1, 7, 8, 9},
+                             rows_per_step=640, full_steps=(23,))
     print("config 5 worst max-abs %.3g rel-L2 %.3g" % worst)
+
+
+def _variable_chunk_cfg(D: int, pinned: int) -> dict:
+    split = dict(rope_t=32, rope_h=48, rope_w=48) if D == 128 else dict(rope_t=16, rope_h=24, rope_w=24)
+    return dict(name="variable chunks", n_layers=2, n_heads=3, head_dim=D, grid_h=8, grid_w=22,
+                max_frames_per_chunk=4, window_frames=5, pinned_frames=pinned, steps=12,
+                dist="outlier_channels", rope_base=10000.0, **split)
+
+
+@pytest.mark.parametrize("D", [128, 64])
+@pytest.mark.parametrize("pinned", [0, 1])
+def test_chunks_of_one_to_four_frames(gpu, D, pinned):
+    """F_max = 4: chunk steps stage 1, 2, 3, 4, 3, 1, 4, 2, ... frames (so the
+    ring's slots are reused at every offset), with and without the pinned
+    conditioning slot, at a token count (176) that is not a multiple of the
+    128-row or 64-key tiles; the whole attention output and every append is
+    compared at every step."""
+    cfg = _variable_chunk_cfg(D, pinned)
+    pattern = [1, 2, 3, 4, 3, 1, 4, 2, 2, 4, 1, 3]
+    R = Runner(2, cfg)
+    worst = 0.0
+    if pinned:
+        for layer in range(2):
+            R.append(layer, -1, 1)
+        for layer in range(2):
+            g, o = R.attend(layer)
+            mx, rl = attn_errors(g, o)
+            assert mx <= ATOL_MAX and rl <= REL_L2, (D, "pinned chunk", layer, mx, rl)
+        R.advance()
+    for step, F in enumerate(pattern):
+        for layer in range(2):
+            R.append(layer, step, F)
+        for layer in range(2):
+            g, o = R.attend(layer)
+            mx, rl = attn_errors(g, o)
+            worst = max(worst, mx)
+            assert mx <= ATOL_MAX and rl <= REL_L2, (D, pinned, step, F, layer, mx, rl)
+        R.advance()
+    R.cache.close()
+    print(f"F_max 4, D {D}, pinned {pinned}: worst max-abs {worst:.3g}")
+
+
+def test_several_denoising_passes_per_chunk(gpu):
+    """Several append + attend passes per chunk before one advance (each pass
+    with new Q/K/V for the same frames): every pass's append and output match
+    the oracle driven through the same passes, and the advance commits the
+    last pass's K/V."""
+    cfg = configs.get(2)
+    R = Runner(2, cfg)
+    for step in range(cfg["window_frames"] + 3):
+        for p in range(3):
+            for layer in range(cfg["n_layers"]):
+                R.append(layer, 100 * p + step, 1)
+            for layer in range(cfg["n_layers"]):
+                g, o = R.attend(layer)
+                mx, rl = attn_errors(g, o)
+                assert mx <= ATOL_MAX and rl <= REL_L2, (step, p, layer, mx, rl)
+        R.advance()
+    R.cache.close()
 
 
 def test_full_shape_48_layer_sequence(gpu):
