@@ -13,15 +13,20 @@ above L2 too.
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
     python bench.py --workload seq48 [--steps K] [--warmup W]
 
---workload seq48 times the 48-layer step at the same shape instead (every
-layer appended and attended, then one advance; the ring full), reporting ms
-per step and the spread of the per-layer times; it prints a line of its own
-and is not the headline metric.
+On one GPU the same JSON line also carries, under "workloads", the other
+full-shape workloads timed on their own: the long-window layer (2 frames per
+chunk, W = 16 plus the pinned slot), three denoising passes per chunk, and
+the 48-layer step (every layer appended and attended, then one advance) with
+the spread of its per-layer times.  --workload seq48 prints only the latter.
+
+"e2e" is the same layer-step through the public API with the inputs copied
+from pinned host memory and the output copied back every step, the copies on
+their own streams so that they overlap the kernels of neighbouring steps.
 
 N > 1 runs N independent replicas (one per GPU, launched by torchrun); the
 path has no data exchange, the process group only carries the barrier and
 the max-over-ranks of the timed region.  --impl reference times the CPU
-oracle on a bounded sample of the same workload on the host cores.
+oracle on whole layer-steps of the same workload on the host cores.
 """
 from __future__ import annotations
 
@@ -56,7 +61,7 @@ def workload(cfg):
     T = cfg["grid_h"] * cfg["grid_w"]
     H, D, W, F = cfg["n_heads"], cfg["head_dim"], cfg["window_frames"], cfg["max_frames_per_chunk"]
     M = F * T
-    N = (W + F) * T
+    N = (cfg["pinned_frames"] + W + F) * T
     flops = 4.0 * M * N * D * H               # QK^T + PV, algorithmic
     append_bytes = (3 * 2 * D + 3 * D + 12) * M * H   # bf16 in, codes + 3 fp32 scales out
     return dict(T=T, H=H, D=D, M=M, N=N, flops=flops, append_bytes=append_bytes)
@@ -136,18 +141,18 @@ class ClockSampler:
 
 
 class OracleTimer:
-    """The CPU oracle, as it stands, timed on bounded samples of one
-    full-shape layer-step: the ring holds W committed frames (their codes are
-    synthetic and not timed); each sample times the oracle's append of
-    `r_app` token rows of Q, K and V (all heads), its fp64 attention for
-    `r_att` query rows (all heads) over the full key set, and the ring
-    update, and extrapolates each part linearly to the whole step."""
+    """The CPU oracle, as it stands, timed on whole layer-steps of the
+    full-shape workload: the ring holds W committed frames (their codes are
+    synthetic and not timed), and each step times the oracle's append of all
+    T token rows of Q, K and V (all heads, the C oracle), its fp64 attention
+    of every query row of every head over the full key set (the oracle's
+    library-matmul form of the definition) and the ring advance."""
 
     def __init__(self, cfg):
         import numpy as np
         import oracle
         from kv_cache_serving_append_b200 import synth
-        self.np, self.oracle, self.cfg = np, oracle, cfg
+        self.np, self.oracle, self.synth, self.cfg = np, oracle, synth, cfg
         self.wl = workload(cfg)
         self.ora = oracle.OracleCache(cfg)
         rng = np.random.default_rng(0)
@@ -160,52 +165,27 @@ class OracleTimer:
             L["sv"][s] = 0.01
             L["staged"] = 1
             self.ora.advance()
-        q, k, v = synth.chunk(CFG_ID, cfg, 0, 0, 1)
-        self.bits = [synth.bf16_bits(t) for t in (q, k, v)]
-        self.ora.append(0, *self.bits, 1)
-        self.split = (cfg["rope_t"], cfg["rope_h"], cfg["rope_w"])
+        self.inputs = []
+        for i in range(2):
+            q, k, v = synth.chunk(CFG_ID, cfg, 0, 100 + i, 1)
+            self.inputs.append([synth.bf16_bits(t) for t in (q, k, v)])
 
-    def sample(self, r_app: int, r_att: int, h_s: int, offset: int = 0):
-        """µs for the whole layer-step, extrapolated from timed pieces.
-
-        Attention is timed on h_s heads for r_att and then 2*r_att query
-        rows; the difference is the per-row cost and the rest the per-call
-        cost of dequantising the key set, so that
-            t_attn = (H / h_s) * (t_call + (M / r_att) * t_rows).
-        """
-        np, oracle, wl = self.np, self.oracle, self.wl
-        T, M, H = wl["T"], wl["M"], wl["H"]
-        r0 = (offset * r_app) % (T - r_app + 1)
+    def step(self, i: int) -> float:
+        """Seconds for one whole layer-step (append, attention, advance)."""
         t0 = time.perf_counter()
-        for i, x in enumerate(self.bits):
-            oracle.append_tensor(np.ascontiguousarray(x[r0:r0 + r_app]), r_app,
-                                 self.cfg["grid_w"], 8, i < 2, self.split)
-        t1 = time.perf_counter()
-        L = self.ora.layers[0]
-        h0 = (offset * h_s) % (H - h_s + 1)
-        hs = slice(h0, h0 + h_s)
-        _, kc, sk, vc, sv = self.ora.key_set(0)
-        args = (L["qc"][hs], L["sq"][hs], kc[hs], sk[hs], vc[hs], sv[hs])
-        times = []
-        for r in (r_att, 2 * r_att):
-            rows = ((np.arange(r) * 997 + offset * 131) % M).astype(np.int32)
-            ta = time.perf_counter()
-            oracle.attend(*args, rows=rows)
-            times.append(time.perf_counter() - ta)
-        t_rows = max(times[1] - times[0], 1e-9)
-        t_call = max(times[0] - t_rows, 0.0)
-        t2 = time.perf_counter()
-        ring = oracle.OracleRing(self.cfg["window_frames"], 1, 0)
-        for _ in range(self.cfg["window_frames"] + 1):
-            ring.commit(1)
-        t3 = time.perf_counter()
-        attn_s = (H / h_s) * (t_call + (M / r_att) * t_rows)
-        us = ((t1 - t0) * T / r_app + attn_s + (t3 - t2) / (self.cfg["window_frames"] + 1)) * 1e6
-        desc = (f"oracle on one full-shape layer-step, sampled: append of {r_app} of {T} token "
-                f"rows (Q, K, V, all {H} heads), fp64 attention of {h_s} of {H} heads for "
-                f"{r_att} and {2 * r_att} of {M} query rows over {wl['N']} keys (per-row and "
-                f"per-call costs separated), each extrapolated linearly to the full step")
-        return us, desc
+        self.ora.append(0, *self.inputs[i % 2], 1)
+        out = self.ora.attend(0, matmul=True)
+        self.ora.advance()
+        dt = time.perf_counter() - t0
+        assert out.shape == (self.wl["M"], self.wl["H"], self.wl["D"])
+        return dt
+
+    def describe(self) -> str:
+        wl = self.wl
+        return (f"full layer-step: oracle append of all {wl['T']} token rows of Q, K and V "
+                f"({wl['H']} heads, plain C), fp64 attention of all {wl['M']} query rows x "
+                f"{wl['H']} heads over {wl['N']} keys (the oracle's library-matmul form: "
+                f"PyTorch CPU float64), ring advance; timed, not extrapolated")
 
 
 def max_over_ranks(value_ms: float, world: int, device) -> float:
@@ -225,16 +205,15 @@ def us_per_layer_step(elapsed_ms: float, steps: int, world: int) -> float:
     return elapsed_ms * 1e3 / (steps * world)
 
 
-def run_seq48(args):
-    """48 layers x (append + attend), then advance, per step; one GPU."""
+def run_seq48_timing(dev, steps: int, warmup: int) -> dict:
+    """48 layers x (append + attend), then advance, per step, ring full; the
+    step time and the spread of the per-layer (append + attend) times."""
     import torch
     from kv_cache_serving_append_b200 import configs, rtv, synth
     cfg = configs.get(4)
     wl = workload(cfg)
     L = cfg["n_layers"]
-    dev = torch.device("cuda", 0)
-    torch.cuda.set_device(dev)
-    cache = rtv.Cache(cfg)
+    cache = rtv.Cache(cfg, dev)
     sets = [synth.chunk(4, cfg, 0, 100 + i, 1, device=dev) for i in range(N_INPUT_SETS)]
     out = torch.empty((wl["T"], wl["H"], wl["D"]), dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
@@ -251,63 +230,73 @@ def run_seq48(args):
         if cache.advance():
             raise RuntimeError("advance failed")
 
-    for i in range(cfg["window_frames"] + 1 + args.warmup):   # fill the ring, warm up
+    for i in range(cfg["window_frames"] + 1 + warmup):   # fill the ring, warm up
         step(i)
     torch.cuda.synchronize()
     evs = [[[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(L)]
-           for _ in range(args.steps)]
+           for _ in range(steps)]
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
     t0.record(stream)
-    for i in range(args.steps):
+    for i in range(steps):
         step(i, evs[i])
     t1.record(stream)
     torch.cuda.synchronize()
     if cache.poll_error():
         raise RuntimeError("kernel error in the timed region")
-    ms = t0.elapsed_time(t1) / args.steps
-    per_layer = [statistics.mean(evs[i][l][0].elapsed_time(evs[i][l][1]) for i in range(args.steps)) * 1e3
+    ms = t0.elapsed_time(t1) / steps
+    per_layer = [statistics.mean(evs[i][l][0].elapsed_time(evs[i][l][1]) for i in range(steps)) * 1e3
                  for l in range(L)]
-    line = {"metric": "ms per 48-layer step (append+attn per layer, then advance) at full shape",
-            "value": ms, "unit": "ms/step", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
-            "higher_is_better": False, "data": "synthetic",
-            "config": {"workload": "48 layers x (append + attend), 40 heads x D128, 2992 tokens/frame, "
-                                   "W=8, ring full", "cache_bytes": cache.nbytes},
-            "per_layer_us": {"mean": statistics.mean(per_layer), "stdev": statistics.pstdev(per_layer),
-                             "min": min(per_layer), "max": max(per_layer)},
-            "attend_key_splits": cache.state().last_attend_splits}
+    res = {"workload": "48 layers x (append + attend), 40 heads x D128, 2992 tokens/frame, W=8, "
+                       "ring full, then one advance", "ms_per_step": ms, "steps": steps,
+           "cache_bytes": cache.nbytes,
+           "per_layer_us": {"mean": statistics.mean(per_layer), "stdev": statistics.pstdev(per_layer),
+                            "min": min(per_layer), "max": max(per_layer)},
+           "attend_key_splits": cache.state().last_attend_splits}
     cache.close()
+    return res
+
+
+def run_seq48(args):
+    """--workload seq48: the 48-layer step on its own JSON line (one GPU)."""
+    import torch
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    r = run_seq48_timing(dev, args.steps, args.warmup)
+    line = {"metric": "ms per 48-layer step (append+attn per layer, then advance) at full shape",
+            "value": r["ms_per_step"], "unit": "ms/step", "n_gpus": 1, "steps": args.steps,
+            "warmup": args.warmup, "higher_is_better": False, "data": "synthetic",
+            "config": {"workload": r["workload"], "cache_bytes": r["cache_bytes"]},
+            "per_layer_us": r["per_layer_us"], "attend_key_splits": r["attend_key_splits"]}
     print(json.dumps(line))
     return 0
 
 
 def run_reference(args):
-    """--impl reference: the CPU oracle as it stands, on the host cores."""
+    """--impl reference: the CPU oracle as it stands, on the host cores, one
+    whole full-shape layer-step per step (rank 0 only)."""
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
     import oracle
+    import torch
     from kv_cache_serving_append_b200 import configs
     cfg = configs.get(CFG_ID)
     timer = OracleTimer(cfg)
-    n = args.warmup + args.steps
-    # bound the whole run to a few minutes of CPU work: per step, 8 token rows
-    # of the append and 1 head x (n_threads, 2 n_threads) query rows
-    r_att = max(1, oracle.num_threads())
-    vals = []
-    desc = ""
-    for i in range(n):
-        us, desc = timer.sample(8, r_att, 1, offset=i)
-        if i >= args.warmup:
-            vals.append(us)
-    v = statistics.mean(vals)
+    for i in range(args.warmup):
+        timer.step(i)
+    t0 = time.perf_counter()
+    vals = [timer.step(args.warmup + i) for i in range(args.steps)]
+    wall = time.perf_counter() - t0
+    v = statistics.mean(vals) * 1e6
+    cores = max(oracle.num_threads(), torch.get_num_threads())
     line = {"metric": METRIC, "value": v, "unit": "us/layer-step", "impl": "reference",
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
-            "ms_per_step": v / 1000.0, "higher_is_better": False, "scaling": "weak",
-            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "ms_per_step": v / 1000.0, "timed_wall_s": wall, "higher_is_better": False,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": config_block(cfg),
-            "cpu_baseline": {"value": v, "unit": "us/layer-step", "cores": oracle.num_threads(),
-                             "kind": "oracle", "sample": desc},
+            "cpu_baseline": {"value": v, "unit": "us/layer-step", "cores": cores,
+                             "kind": "oracle", "sample": timer.describe()},
             "e2e": {"value": v, "unit": "us/layer-step", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line))
@@ -327,13 +316,203 @@ def config_block(cfg):
             "parallelism": "replicas (one independent cache per GPU)"}
 
 
+def fill_ring(cache, cfg, sets, stream, passes: int = 1):
+    """Append + attend + advance until the ring is full (steady state)."""
+    F = cfg["max_frames_per_chunk"]
+    steps = cfg["window_frames"] // F + 2 + cfg["pinned_frames"]
+    out = torch_empty_out(cfg, cache.device)
+    for i in range(steps):
+        n = 1 if (cfg["pinned_frames"] and i == 0) else F
+        q, k, v = sets[i % len(sets)]
+        rows = n * cfg["grid_h"] * cfg["grid_w"]
+        for _ in range(passes):
+            if cache.append(0, q[:rows], k[:rows], v[:rows], n, stream) or \
+                    cache.attend(0, out[:rows], stream):
+                raise RuntimeError("fill step failed")
+        if cache.advance():
+            raise RuntimeError("advance failed")
+
+
+def torch_empty_out(cfg, device):
+    import torch
+    T = cfg["grid_h"] * cfg["grid_w"]
+    return torch.empty((cfg["max_frames_per_chunk"] * T, cfg["n_heads"], cfg["head_dim"]),
+                       dtype=torch.float32, device=device)
+
+
+def time_layer(cfg_id, dev, steps: int, warmup: int, passes: int = 1, events: bool = True,
+               barrier=None):
+    """Steady-state layer-steps of one workload: per step `passes` x (append +
+    attend), then advance.  Returns device times (ms) per step, per append and
+    per attend (CUDA events on the launching stream) and the split count."""
+    import torch
+    from kv_cache_serving_append_b200 import configs, rtv, synth
+    cfg = configs.get(cfg_id)
+    F = cfg["max_frames_per_chunk"]
+    cache = rtv.Cache(cfg, dev)
+    sets = [synth.chunk(cfg_id, cfg, 0, 100 + i, F, device=dev) for i in range(N_INPUT_SETS)]
+    out = torch_empty_out(cfg, dev)
+    stream = torch.cuda.current_stream(dev)
+    fill_ring(cache, cfg, sets, stream, passes)
+
+    def step(i, ev=None):
+        for p in range(passes):
+            q, k, v = sets[(i * passes + p) % N_INPUT_SETS]
+            if ev is not None:
+                ev[p][0].record(stream)
+            if cache.append(0, q, k, v, F, stream):
+                raise RuntimeError("append failed")
+            if ev is not None:
+                ev[p][1].record(stream)
+            if cache.attend(0, out, stream):
+                raise RuntimeError("attend failed")
+            if ev is not None:
+                ev[p][2].record(stream)
+        if cache.advance():
+            raise RuntimeError("advance failed")
+
+    for i in range(warmup):
+        step(i)
+    torch.cuda.synchronize()
+    if cache.poll_error():
+        raise RuntimeError("kernel error during warm-up")
+    ev = [[[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(passes)]
+          for _ in range(steps)] if events else None
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if barrier:
+        barrier()
+    torch.cuda.synchronize()
+    t0.record(stream)
+    for i in range(steps):
+        step(i, ev[i] if ev else None)
+    t1.record(stream)
+    torch.cuda.synchronize()
+    if barrier:
+        barrier()
+    if cache.poll_error():
+        raise RuntimeError("kernel error in the timed region")
+    res = {"step_ms": t0.elapsed_time(t1) / steps, "splits": cache.state().last_attend_splits,
+           "cache": cache, "sets": sets, "out": out, "cfg": cfg, "stream": stream}
+    if ev:
+        res["append_ms"] = statistics.mean(e[0].elapsed_time(e[1]) for x in ev for e in x)
+        res["attend_ms"] = statistics.mean(e[1].elapsed_time(e[2]) for x in ev for e in x)
+    return res
+
+
+def time_e2e(res, steps: int, warmup: int, world: int, dev):
+    """End to end through the public API, every step: H2D of the step's Q/K/V
+    from pinned host memory, append, attend, D2H of the output.  Copies run on
+    their own streams into double-buffered device inputs and outputs, so the
+    H2D of step i+1 and the D2H of step i-1 overlap step i's kernels; events
+    order every reuse of a buffer.  Timed from the first H2D to the last D2H."""
+    import torch
+    cache, sets, cfg = res["cache"], res["sets"], res["cfg"]
+    stream = res["stream"]
+    F = cfg["max_frames_per_chunk"]
+    h2d_s, d2h_s = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    host_in = [tuple(t.cpu().pin_memory() for t in sets[i]) for i in range(2)]
+    dev_in = [tuple(torch.empty_like(t) for t in sets[0]) for _ in range(2)]
+    dev_out = [torch.empty_like(res["out"]) for _ in range(2)]
+    host_out = [torch.empty(res["out"].shape, dtype=res["out"].dtype).pin_memory() for _ in range(2)]
+    ev = lambda: torch.cuda.Event()   # noqa: E731
+    in_ready = [ev(), ev()]      # H2D into dev_in[b] done
+    in_free = [ev(), ev()]       # append that read dev_in[b] done
+    out_ready = [ev(), ev()]     # attend into dev_out[b] done
+    out_free = [ev(), ev()]      # D2H out of dev_out[b] done
+    for b in range(2):
+        in_free[b].record(stream)
+        out_free[b].record(d2h_s)
+
+    def h2d(i):
+        b = i % 2
+        with torch.cuda.stream(h2d_s):
+            h2d_s.wait_event(in_free[b])
+            for d, h in zip(dev_in[b], host_in[i % 2]):
+                d.copy_(h, non_blocking=True)
+            in_ready[b].record(h2d_s)
+
+    def compute(i):
+        b = i % 2
+        stream.wait_event(in_ready[b])
+        if cache.append(0, *dev_in[b], F, stream):
+            raise RuntimeError("e2e append failed")
+        in_free[b].record(stream)
+        stream.wait_event(out_free[b])
+        if cache.attend(0, dev_out[b], stream) or cache.advance():
+            raise RuntimeError("e2e attend failed")
+        out_ready[b].record(stream)
+
+    def d2h(i):
+        b = i % 2
+        with torch.cuda.stream(d2h_s):
+            d2h_s.wait_event(out_ready[b])
+            host_out[b].copy_(dev_out[b], non_blocking=True)
+            out_free[b].record(d2h_s)
+
+    def run(n):
+        h2d(0)
+        for i in range(n):
+            if i + 1 < n:
+                h2d(i + 1)
+            compute(i)
+            d2h(i)
+
+    run(warmup)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(h2d_s)
+    run(steps)
+    e1.record(d2h_s)
+    torch.cuda.synchronize()
+    if cache.poll_error():
+        raise RuntimeError("kernel error in the end-to-end region")
+    ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
+    h2d_bytes = sum(t.numel() * t.element_size() for t in dev_in[0])
+    d2h_bytes = host_out[0].numel() * host_out[0].element_size()
+    return ms / steps, h2d_bytes, d2h_bytes
+
+
+def extra_workloads(dev, steps: int, warmup: int):
+    """The other full-shape workloads, each timed on its own (one GPU)."""
+    import torch
+    out = {}
+    k = max(3, min(steps, 10))
+    # long window: 2 frames per chunk, W = 16, pinned conditioning slot
+    r = time_layer(5, dev, k, 3)
+    wl = workload(r["cfg"])
+    out["long_window"] = {
+        "workload": "1 layer, 40 heads x D128, 2992 tokens/frame, 2 frames/chunk, W=16 + pinned "
+                    "slot, steady state", "us_per_layer_step": r["step_ms"] * 1e3,
+        "append_us": r["append_ms"] * 1e3, "attn_us": r["attend_ms"] * 1e3,
+        "attn_tflops": wl["flops"] / (r["attend_ms"] * 1e-3) / 1e12,
+        "append_gbs": wl["append_bytes"] / (r["append_ms"] * 1e-3) / 1e9,
+        "keys_per_query": wl["N"], "attend_key_splits": r["splits"], "steps": k}
+    r["cache"].close()
+    del r
+    # several denoising passes per chunk (3 x append + attend, then advance)
+    r = time_layer(CFG_ID, dev, k, 3, passes=3)
+    out["multipass"] = {
+        "workload": "full-shape layer, 3 denoising passes per chunk (append + attend each), "
+                    "then one advance", "us_per_chunk": r["step_ms"] * 1e3,
+        "us_per_pass": r["step_ms"] * 1e3 / 3, "append_us": r["append_ms"] * 1e3,
+        "attn_us": r["attend_ms"] * 1e3, "steps": k}
+    r["cache"].close()
+    del r
+    torch.cuda.empty_cache()
+    out["seq48"] = run_seq48_timing(dev, min(steps, 5), 2)
+    torch.cuda.empty_cache()
+    return out
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=1500)
-    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extra", action="store_true",
+                    help="skip the long-window, multi-pass and 48-layer workloads")
     ap.add_argument("--workload", default="layer", choices=["layer", "seq48"])
     args = ap.parse_args()
     if args.impl == "reference":
@@ -352,101 +531,27 @@ def main():
         from datetime import timedelta
         dist.init_process_group("nccl", device_id=dev, timeout=timedelta(seconds=120))
 
-    from kv_cache_serving_append_b200 import configs, rtv, synth
+    from kv_cache_serving_append_b200 import configs
     cfg = configs.get(CFG_ID)
     wl = workload(cfg)
-    T, H, D = wl["T"], wl["H"], wl["D"]
-    cache = rtv.Cache(cfg, dev)
-    sets = [synth.chunk(CFG_ID, cfg, 0, 100 + i, 1, device=dev) for i in range(N_INPUT_SETS)]
-    # fp32 output: the configuration the parity tests hold to the tolerance
-    out = torch.empty((T, H, D), dtype=torch.float32, device=dev)
-    stream = torch.cuda.current_stream(dev)
-
-    def step(i):
-        q, k, v = sets[i % N_INPUT_SETS]
-        st = cache.append(0, q, k, v, 1, stream)
-        if st:
-            raise rtv.RtvError(st, "append")
-        st = cache.attend(0, out, stream)
-        if st:
-            raise rtv.RtvError(st, "attend")
-        st = cache.advance()
-        if st:
-            raise rtv.RtvError(st, "advance")
-
-    # fill the ring (steady state), then warm up
-    for i in range(cfg["window_frames"] + 1 + args.warmup):
-        step(i)
-    torch.cuda.synchronize()
-    if cache.poll_error():
-        raise RuntimeError("kernel error during warm-up")
-
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
-    t_start = torch.cuda.Event(enable_timing=True)
-    t_end = torch.cuda.Event(enable_timing=True)
     sampler = ClockSampler(torch.cuda.get_device_properties(dev)) if rank == 0 else None
+    # time_layer fills the ring and runs the warm-up steps, then times exactly
+    # `steps` steps between a barrier + synchronize on each side
     if sampler:
         sampler.start()
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize()
-    t_start.record(stream)
-    for i in range(args.steps):
-        q, k, v = sets[i % N_INPUT_SETS]
-        e = ev[i]
-        e[0].record(stream)
-        if cache.append(0, q, k, v, 1, stream):
-            raise RuntimeError("append failed")
-        e[1].record(stream)
-        if cache.attend(0, out, stream):
-            raise RuntimeError("attend failed")
-        e[2].record(stream)
-        if cache.advance():
-            raise RuntimeError("advance failed")
-    t_end.record(stream)
-    torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
+    res = time_layer(CFG_ID, dev, args.steps, args.warmup,
+                     barrier=dist.barrier if world > 1 else None)
     clocks = sampler.stop() if sampler else None
-    if cache.poll_error():
-        raise RuntimeError("kernel error in the timed region")
-    elapsed_ms = max_over_ranks(t_start.elapsed_time(t_end), world, dev)
-    # kernels per step: append, attention, and the split merge when the key range is split
-    splits = cache.state().last_attend_splits
+    elapsed_ms = max_over_ranks(res["step_ms"] * args.steps, world, dev)
+    splits = res["splits"]
     launches_per_step = 2 + (1 if splits > 1 else 0)
-    append_ms = statistics.mean(ev[i][0].elapsed_time(ev[i][1]) for i in range(args.steps))
-    attend_ms = statistics.mean(ev[i][1].elapsed_time(ev[i][2]) for i in range(args.steps))
+    append_ms, attend_ms = res["append_ms"], res["attend_ms"]
 
-    # end to end through the public API: pinned host inputs -> H2D -> append ->
-    # attend -> D2H of the output, every step
-    host_in = [tuple(t.cpu().pin_memory() for t in sets[i]) for i in range(2)]
-    dev_in = tuple(torch.empty_like(t) for t in sets[0])
-    host_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-    e2e_steps = max(20, min(200, args.steps // 5))
-
-    def e2e_step(i):
-        hq = host_in[i % 2]
-        for d, h in zip(dev_in, hq):
-            d.copy_(h, non_blocking=True)
-        if cache.append(0, *dev_in, 1, stream) or cache.attend(0, out, stream) or cache.advance():
-            raise RuntimeError("e2e step failed")
-        host_out.copy_(out, non_blocking=True)
-
-    for i in range(5):
-        e2e_step(i)
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize()
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for i in range(e2e_steps):
-        e2e_step(i)
-    e1.record(stream)
-    torch.cuda.synchronize()
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
-    h2d = sum(t.numel() * t.element_size() for t in dev_in)
-    d2h = host_out.numel() * host_out.element_size()
+    e2e_steps = max(20, min(200, args.steps))
+    e2e_ms, h2d, d2h = time_e2e(res, e2e_steps, 5, world, dev)
+    res["cache"].close()
+    del res
+    torch.cuda.empty_cache()
 
     hbm_gbs, bf16_tf, bf16_tf_sus, peak_src = load_peaks()
     fp8_peak = 2.0 * bf16_tf
@@ -471,21 +576,26 @@ def main():
         "roofline_append": {"kernel": "rtv append (fused RoPE+amax+E4M3)", "bound": "hbm",
                             "achieved": append_gbs, "peak": hbm_gbs, "unit": "GB/s",
                             "frac": append_gbs / hbm_gbs,
+                            "peak_source": f"{peak_src} HBM copy",
                             "traffic": ncu_traffic("append_kernel.cu", "append_full_shape_ncu.md"),
                             "algorithmic_bytes_per_launch": wl["append_bytes"]},
-        "e2e": {"value": e2e_ms * 1e3 / (e2e_steps * world), "unit": "us/layer-step",
-                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "e2e": {"value": e2e_ms * 1e3 / world, "unit": "us/layer-step",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "overlap": "H2D of step i+1 and D2H of step i-1 on their own streams beside "
+                           "step i's kernels (double-buffered device inputs and outputs)"},
         "gpu_launches": launches_per_step * args.steps,
         "attend_key_splits": splits,
         "clocks": clocks,
     }
+    if world == 1 and not args.no_extra:
+        line["workloads"] = extra_workloads(dev, args.steps, args.warmup)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         import oracle
         timer = OracleTimer(cfg)
-        us, desc = timer.sample(r_app=256, r_att=2 * oracle.num_threads(), h_s=4)
+        us = timer.step(0) * 1e6
         line["cpu_baseline"] = {"value": us, "unit": "us/layer-step",
-                                "cores": oracle.num_threads(), "kind": "oracle", "sample": desc}
-    cache.close()
+                                "cores": max(oracle.num_threads(), torch.get_num_threads()),
+                                "kind": "oracle", "sample": timer.describe()}
     if rank == 0:
         print(json.dumps(line))
     if world > 1:
