@@ -257,6 +257,53 @@ def run_seq48_timing(dev, steps: int, warmup: int) -> dict:
     return res
 
 
+def run_seq48_graph_timing(dev, steps: int, warmup: int) -> dict:
+    """The same 48-layer step replayed from one captured CUDA graph (ring
+    state on the device; rtv_step_graph_*): one launch per step."""
+    import torch
+    from kv_cache_serving_append_b200 import configs, rtv, synth
+    cfg = configs.get(4)
+    wl = workload(cfg)
+    L = cfg["n_layers"]
+    cache = rtv.Cache(cfg, dev)
+    sets = [synth.chunk(4, cfg, 0, 100 + i, 1, device=dev) for i in range(N_INPUT_SETS)]
+    out = torch.empty((wl["T"], wl["H"], wl["D"]), dtype=torch.float32, device=dev)
+    stream = torch.cuda.Stream(dev)
+    with torch.cuda.stream(stream):
+        for i in range(cfg["window_frames"]):          # direct calls fill the window
+            for layer in range(L):
+                q, k, v = sets[(i * L + layer) % N_INPUT_SETS]
+                if cache.append(layer, q, k, v, 1, stream) or cache.attend(layer, out, stream):
+                    raise RuntimeError("append/attend failed")
+            if cache.advance():
+                raise RuntimeError("advance failed")
+        g = rtv.StepGraph(cache, 1, [sets[l % N_INPUT_SETS][0] for l in range(L)],
+                          [sets[l % N_INPUT_SETS][1] for l in range(L)],
+                          [sets[l % N_INPUT_SETS][2] for l in range(L)], [out] * L, stream)
+        for _ in range(warmup):
+            if g.launch(stream):
+                raise RuntimeError("graph launch failed")
+        stream.synchronize()
+        t0 = torch.cuda.Event(enable_timing=True)
+        t1 = torch.cuda.Event(enable_timing=True)
+        t0.record(stream)
+        host0 = time.perf_counter()
+        for _ in range(steps):
+            if g.launch(stream):
+                raise RuntimeError("graph launch failed")
+        host_us = (time.perf_counter() - host0) * 1e6 / steps
+        t1.record(stream)
+        stream.synchronize()
+    if cache.poll_error():
+        raise RuntimeError("kernel error in the timed region")
+    res = {"workload": "48 layers x (append + attend) + device ring advance, one CUDA graph "
+                       "launch per step, ring full", "ms_per_step": t0.elapsed_time(t1) / steps,
+           "host_us_per_launch": host_us, "steps": steps}
+    g.close()
+    cache.close()
+    return res
+
+
 def run_seq48(args):
     """--workload seq48: the 48-layer step on its own JSON line (one GPU)."""
     import torch
@@ -500,6 +547,8 @@ def extra_workloads(dev, steps: int, warmup: int):
     del r
     torch.cuda.empty_cache()
     out["seq48"] = run_seq48_timing(dev, min(steps, 5), 2)
+    torch.cuda.empty_cache()
+    out["seq48_graph"] = run_seq48_graph_timing(dev, min(steps, 5), 2)
     torch.cuda.empty_cache()
     return out
 

@@ -48,7 +48,8 @@ typedef enum {
     RTV_ERR_CUDA = 3,        /* a CUDA runtime/driver call failed */
     RTV_ERR_STATE = 4,       /* call not valid in the cache's current state */
     RTV_ERR_TIMEOUT = 5,     /* a kernel's bounded wait ran out (see rtv_poll_error) */
-    RTV_ERR_UNSUPPORTED = 6  /* configuration outside what the kernels implement */
+    RTV_ERR_UNSUPPORTED = 6, /* configuration outside what the kernels implement */
+    RTV_ERR_BOUNDS = 7       /* a debug build's kernel found a slot index out of range */
 } rtv_status;
 
 /* Output element types of rtv_attend. */
@@ -231,6 +232,51 @@ rtv_status rtv_attend(rtv_cache* cache, int layer, void* out, int out_dtype, voi
  */
 rtv_status rtv_cache_advance(rtv_cache* cache);
 
+/*
+ * Whole-step CUDA graph with the ring state resident on the device.
+ * Source: lhc.media, "Runway partage la construction de Runway Characters",
+ * third paragraph (CUDA graphs among the serving optimisations); aidose.in,
+ * "Runway explains how it serves a 57B video model in real time", fourth
+ * paragraph (one host synchronisation per step cost 168.5 -> 278 ms): the
+ * host should only launch, never wait, and launch as little as possible.
+ *
+ * rtv_step_graph_create captures one steady-state step of every layer --
+ * rtv_cache_append then rtv_attend for layers 0..n_layers-1, then a one-warp
+ * kernel that advances the ring state held in the cache buffer -- into one
+ * CUDA graph.  The captured kernels read the staged and key-set slots, the
+ * frame-axis RoPE cos/sin and the V-scale tag from that device state instead
+ * of their launch parameters, so the same graph serves every later step.
+ *   n_frames      frames per chunk, 1..max_frames_per_chunk
+ *   q, k, v       arrays of n_layers device pointers: each layer's bf16
+ *                 [n_frames*T][n_heads][head_dim] inputs; the graph reads
+ *                 whatever these buffers hold when it runs, so the caller
+ *                 writes each step's Q/K/V into them (stream-ordered) before
+ *                 rtv_step_graph_launch
+ *   out           array of n_layers device pointers, each layer's output as
+ *                 for rtv_attend (out_dtype RTV_OUT_F32 or RTV_OUT_BF16)
+ *   stream        a non-NULL stream: used for the capture (legacy-stream
+ *                 capture is not allowed); synchronised once
+ * Requires the steady state: the pinned frame committed (when configured),
+ * at least window_frames generated frames committed, no layer staged.  The
+ * caller keeps the buffers alive until rtv_step_graph_destroy.
+ * Errors: RTV_ERR_INVALID_ARG, RTV_ERR_STATE (not steady), RTV_ERR_CUDA,
+ * RTV_ERR_OOM.
+ *
+ * rtv_step_graph_launch enqueues one step on `stream` (no host
+ * synchronisation) and makes the same step in the host ring state (as
+ * rtv_cache_advance would after every layer's append), so rtv_cache_get_state
+ * and direct calls stay consistent.  Direct append/attend/advance calls may
+ * be mixed in between: if they moved the ring, the launch first copies the
+ * current state to the device (stream-ordered).  Errors: RTV_ERR_INVALID_ARG,
+ * RTV_ERR_STATE (a layer is staged by a direct call), RTV_ERR_CUDA.
+ */
+typedef struct rtv_step_graph rtv_step_graph;
+rtv_status rtv_step_graph_create(rtv_cache* cache, int n_frames, const void* const* q,
+                                 const void* const* k, const void* const* v, void* const* out,
+                                 int out_dtype, void* stream, rtv_step_graph** graph);
+rtv_status rtv_step_graph_launch(rtv_step_graph* graph, void* stream);
+rtv_status rtv_step_graph_destroy(rtv_step_graph* graph);
+
 /* Ring state (host-side; no device access). */
 rtv_status rtv_cache_get_state(const rtv_cache* cache, rtv_cache_state* out);
 
@@ -262,7 +308,7 @@ rtv_status rtv_poll_error(rtv_cache* cache);
 /*
  * The key-range split rtv_attend chooses (host arithmetic only; no device
  * needed).  n_units = ceil(n_frames*T / 256) * n_heads CTAs of one key range
- * each, n_kv_tiles = key frames * ceil(T / 64), sm_count = the device's SMs.
+ * each, n_kv_tiles = key frames * ceil(T / 128), sm_count = the device's SMs.
  * Out: n_split in 1..4 and tiles_per_split (the last split may hold fewer,
  * none is empty).  The plan minimises ceil(n_units*s / sm_count) / s plus 3%
  * per extra split, with at least 8 KV tiles per split.
@@ -305,6 +351,19 @@ rtv_status rtv_attend_static_scratch(rtv_cache* cache, int layer, void* out, int
  * about one second).  Used only by the failure-detection test.
  */
 rtv_status rtv_debug_set_wait_fault(rtv_cache* cache, int enable, long long wait_limit_cycles);
+
+/*
+ * Debug builds (librtv_debug.so, compiled with RTV_DEBUG): every kernel
+ * checks the ring slots it is given against the cache's slot count before it
+ * touches memory; a launch that finds one out of range records it in the
+ * device error word and returns, and rtv_poll_error then reports
+ * RTV_ERR_BOUNDS.  rtv_debug_build returns 1 in such a build, 0 otherwise.
+ * rtv_debug_corrupt_next_attend makes the next rtv_attend name slot
+ * `bad_slot` first in its key set (the test of that check); it returns
+ * RTV_ERR_UNSUPPORTED in a release build, where nothing would catch it.
+ */
+int rtv_debug_build(void);
+rtv_status rtv_debug_corrupt_next_attend(rtv_cache* cache, int bad_slot);
 
 #ifdef __cplusplus
 }

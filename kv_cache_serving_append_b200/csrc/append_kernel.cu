@@ -8,17 +8,23 @@
 // (fixed fp32 rounding order, RNE saturating E4M3, reciprocal multiply) is the
 // library's definition, restated in rtv.h.
 //
-// Work split: one block = up to rows_per_block token rows of one frame times
-// all heads, for one of Q/K/V (blockIdx.y).  A (row, head) item is 2*D bytes
-// of bf16, handled by a half-warp: each of the 16 lanes loads D/16 contiguous
-// elements (16 bytes at D=128), so every input byte is read once with full
-// 32-byte sectors, and writes D/16 codes (8 bytes), so the 16 lanes write one
-// contiguous D-byte row of codes.  The rotate-half partner of a lane's
-// elements sits 2 lanes away in the frame segment and 3 lanes away in the row
-// and column segments (for the supported splits), fetched with a shuffle.
-// Each group keeps ITEMS loads in flight to cover HBM latency.
+// Work split: blockIdx.y picks Q, K or V; a half-warp (16 lanes) owns one
+// token row at a time (grid-stride over the chunk's rows) and walks that
+// row's heads.  A (row, head) item is 2*D bytes of bf16: lane i loads D/16
+// contiguous elements (16 bytes at D = 128), so the 16 lanes read the item in
+// full 32-byte sectors, and the H items of a row are one contiguous stretch
+// of memory.  The RoPE cos/sin a lane needs depend only on the row (its
+// frame, grid row and grid column) and on the lane's place in head_dim, so
+// they are loaded into registers once per row and reused for every head.
+// The rotate-half partner of a lane's elements sits 2 lanes away in the frame
+// segment and 3 lanes away in the grid-row and grid-column segments (for the
+// supported splits), fetched with a shuffle.  Each half-warp keeps kItems
+// loads in flight: the load of head h + kItems is issued as soon as head h is
+// done.  Every input byte is read once and every code byte written once.
 #include <cuda_bf16.h>
 #include <cuda_fp8.h>
+
+#include <mutex>
 
 #include "rtv_internal.h"
 
@@ -26,8 +32,8 @@ namespace rtv {
 namespace {
 
 constexpr int kThreads = 256;
-constexpr int kGroups = kThreads / 16;   // half-warps per block
-constexpr int kItems = 4;                // items in flight per half-warp
+constexpr int kGroups = kThreads / 16;   // half-warps (rows in flight) per block
+constexpr int kItems = 3;                // loads in flight per half-warp
 
 template <int E>
 struct Vec;
@@ -68,6 +74,8 @@ __device__ __forceinline__ uint2 shfl_vec(const uint2& v, int src)
     r.y = __shfl_sync(0xffffffffu, v.y, src);
     return r;
 }
+__device__ __forceinline__ uint4 xor_vec(const uint4& v, uint32_t m) { return make_uint4(v.x ^ m, v.y ^ m, v.z ^ m, v.w ^ m); }
+__device__ __forceinline__ uint2 xor_vec(const uint2& v, uint32_t m) { return make_uint2(v.x ^ m, v.y ^ m); }
 
 // E4M3 round-to-nearest-even with saturation to +-448 (hardware cvt).
 __device__ __forceinline__ uint16_t e4m3x2(float lo, float hi)
@@ -94,73 +102,41 @@ __device__ __forceinline__ void store_codes<4>(uint8_t* dst, const float* y, flo
     *reinterpret_cast<uint32_t*>(dst) = w0;
 }
 
-constexpr int kMaxRows = 32;   // token rows per block (host keeps rows_per_block <= this)
-
+// E consecutive floats from a 16-byte aligned address.
 template <int E>
 __device__ __forceinline__ void load_vec(const float* p, float* x)
 {
 #pragma unroll
     for (int i = 0; i < E; i += 4) {
-        const float4 v = *reinterpret_cast<const float4*>(p + i);
+        const float4 v = __ldg(reinterpret_cast<const float4*>(p + i));
         x[i] = v.x; x[i + 1] = v.y; x[i + 2] = v.z; x[i + 3] = v.w;
     }
 }
 
-__device__ __forceinline__ uint4 xor_vec(const uint4& v, uint32_t m) { return make_uint4(v.x ^ m, v.y ^ m, v.z ^ m, v.w ^ m); }
-__device__ __forceinline__ uint2 xor_vec(const uint2& v, uint32_t m) { return make_uint2(v.x ^ m, v.y ^ m); }
-
-// D = head_dim, E = D / 16 elements per lane.
-template <int D>
-__global__ void __launch_bounds__(kThreads, 4) append_kernel(const __grid_constant__ AppendParams p)
+// One tensor's rows (Q and K: ROPE; V: not rotated).  D = head_dim, E = D / 16
+// elements per lane.
+template <int D, bool ROPE>
+__device__ __forceinline__ void append_rows(const AppendParams& p, int tensor,
+                                            unsigned int (*s_vmax)[kMaxHeads], float* s_cs)
 {
     constexpr int E = D / 16;
     using V = typename Vec<E>::T;
-    // Per local token row: the RoPE cos/sin this row needs, laid out along
-    // head_dim as [t cos | t sin | h cos | h sin | w cos | w sin] (half-widths).
-    __shared__ __align__(16) float s_tab[kMaxRows][D];
-    __shared__ unsigned int s_vmax[kMaxHeads];
-
-    const int tensor = blockIdx.y;             // 0 = Q, 1 = K, 2 = V
-    const int frame = blockIdx.x / p.blocks_per_frame;
-    const int tok0 = (blockIdx.x % p.blocks_per_frame) * p.rows_per_block;
-    const int n_rows = min(p.rows_per_block, p.T - tok0);
-    const int H = p.H;
-    const int n_items = n_rows * H;
-    const bool rope = tensor != 2;
+    constexpr bool rope = ROPE;
+    const int H = p.H, T = p.T;
+    const int n_rows = p.n_frames * T;
     const int ht = p.n_t / 2, hh = p.n_h / 2, hw = p.n_w / 2;
 
-    for (int i = threadIdx.x; i < H; i += kThreads) s_vmax[i] = 0u;
-    if (rope) {
-        for (int i = threadIdx.x; i < n_rows * D; i += kThreads) {
-            const int r = i / D, d = i - r * D;
-            const int tok = tok0 + r;
-            float v;
-            if (d < 2 * ht) {
-                v = p.t_table[frame][d / ht][d % ht];
-            } else if (d < 2 * ht + 2 * hh) {
-                const int hp = tok / p.grid_w;
-                v = p.h_table[(size_t)hp * 2 * hh + (d - 2 * ht)];
-            } else {
-                const int wp = tok % p.grid_w;
-                v = p.w_table[(size_t)wp * 2 * hw + (d - 2 * ht - 2 * hh)];
-            }
-            s_tab[r][d] = v;
-        }
-    }
-    __syncthreads();
-
     const int lane16 = threadIdx.x & 15;
-    const int group = threadIdx.x >> 4;
     const int lane = threadIdx.x & 31;
 
-    // Fixed per lane: RoPE segment of its E elements, pair index of the
-    // first one, which half of the pair it holds, its partner lane, and where
-    // its cos/sin sit in the row table.
-    int seg_half = ht, seg_lo = 0, tab_lo = 0;
+    // Fixed per lane: RoPE segment of its E elements (0 = frame, 1 = grid
+    // row, 2 = grid column), pair index of the first one, which half of the
+    // pair it holds, and its partner lane.
+    int seg = 0, seg_half = ht, seg_lo = 0;
     if (lane16 * E >= p.n_t + p.n_h) {
-        seg_half = hw; seg_lo = p.n_t + p.n_h; tab_lo = 2 * ht + 2 * hh;
+        seg = 2; seg_half = hw; seg_lo = p.n_t + p.n_h;
     } else if (lane16 * E >= p.n_t) {
-        seg_half = hh; seg_lo = p.n_t; tab_lo = 2 * ht;
+        seg = 1; seg_half = hh; seg_lo = p.n_t;
     }
     const int in_seg = lane16 * E - seg_lo;
     const bool first_half = in_seg < seg_half;
@@ -169,98 +145,204 @@ __global__ void __launch_bounds__(kThreads, 4) append_kernel(const __grid_consta
     // x'[j] = x[j]c - x[j+n/2]s (first half) = x[j]c + (-x[j+n/2])s: the
     // partner's value is negated by flipping its bf16 sign bits (exact).
     const uint32_t neg_partner = first_half ? 0x80008000u : 0u;
-    const int c_off = tab_lo + j0, s_off = tab_lo + seg_half + j0;
 
     const uint16_t* src = p.src[tensor];
-    const int row0 = frame * p.T + tok0;
+    // Rows are visited grid-stride; the trip count is the same for the two
+    // half-warps of a warp only if both have a row, so the loop runs while
+    // either has one (full-warp shuffles need all 32 lanes) and the other
+    // idles through it without memory access.
+    const int stride = gridDim.x * kGroups;
+    const int row_pair0 = blockIdx.x * kGroups + ((threadIdx.x >> 4) & ~1);
+    for (int rbase = row_pair0; rbase < n_rows; rbase += stride) {
+        const int row = rbase + ((threadIdx.x >> 4) & 1);
+        const bool row_ok = row < n_rows;
+        const int frame = row_ok ? row / T : 0;
+        const int tok = row_ok ? row - frame * T : 0;
 
-    // Item it = (row it / H, head it % H), visited with stride kGroups; the
-    // (row, head) pair is advanced incrementally (no division per item).  The
-    // loop bound is taken per warp so the full-warp shuffles always have all
-    // 32 lanes present.
-    int r_it = group / H, h_it = group - (group / H) * H;
-    for (int wbase = group & ~1; wbase < n_items; wbase += kGroups * kItems) {
-        const int base = wbase + (group & 1);
-        V raw[kItems];
-        int rr[kItems], hv[kItems];
+        // this lane's cos/sin for the row, staged in the half-warp's slice of
+        // shared memory (read back per head; 16-byte accesses, no conflicts)
+        float* cs = s_cs + ((threadIdx.x >> 4) * 2 * D) + lane16 * E;   // cos at cs, sin at cs + D
+        if (rope) {
+            float cc[E], ss[E];
+            if (seg == 0) {
+                const float (*tt)[kMaxRopeHalf] = p.ring ? p.ring->t_table[frame] : p.t_table[frame];
 #pragma unroll
-        for (int u = 0; u < kItems; ++u) {
-            rr[u] = r_it;
-            hv[u] = h_it;
-            raw[u] = V{};
-            if (base + u * kGroups < n_items) {
-                const size_t off = ((size_t)(row0 + r_it) * H + h_it) * D + lane16 * E;
-                raw[u] = __ldcs(reinterpret_cast<const V*>(src + off));
-            }
-            h_it += kGroups;
-            while (h_it >= H) { h_it -= H; ++r_it; }
-        }
-#pragma unroll
-        for (int u = 0; u < kItems; ++u) {
-            const bool valid = base + u * kGroups < n_items;
-            const int r = valid ? rr[u] : 0;
-            const int h = hv[u];
-            float y[E];
-            unpack_bf16(raw[u], y);
-            if (rope) {
-                const V praw = xor_vec(shfl_vec(raw[u], partner), neg_partner);
-                float xp[E], cc[E], ss[E];
-                unpack_bf16(praw, xp);
-                load_vec<E>(&s_tab[r][c_off], cc);
-                load_vec<E>(&s_tab[r][s_off], ss);
-#pragma unroll
-                for (int e = 0; e < E; ++e)
-                    y[e] = __fadd_rn(__fmul_rn(y[e], cc[e]), __fmul_rn(xp[e], ss[e]));
-            }
-            float amax = 0.f;
-#pragma unroll
-            for (int e = 0; e < E; ++e) amax = fmaxf(amax, fabsf(y[e]));
-#pragma unroll
-            for (int o = 8; o >= 1; o >>= 1)
-                amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-            if (!valid) continue;
-            const float inv = amax > 0.f ? __fdiv_rn(448.f, amax) : 0.f;
-            const float scale = __fdiv_rn(amax, 448.f);
-            const int tok = tok0 + r;
-            uint8_t* dst;
-            float* sdst;
-            if (tensor == 0) {
-                const size_t qr = (size_t)h * p.q_rows + frame * p.T + tok;
-                dst = p.q_codes + qr * D;
-                sdst = p.q_scales + (size_t)h * p.q_scale_pitch + frame * p.T + tok;
+                for (int e = 0; e < E; ++e) {
+                    cc[e] = tt[0][j0 + e];
+                    ss[e] = tt[1][j0 + e];
+                }
+            } else if (seg == 1) {
+                const float* t = p.h_table + (size_t)(tok / p.grid_w) * 2 * hh;
+                load_vec<E>(t + j0, cc);
+                load_vec<E>(t + hh + j0, ss);
             } else {
-                const size_t sh = (size_t)p.slot[frame] * H + h;
-                dst = p.kv_codes[tensor - 1] + (sh * p.T + tok) * D;
-                sdst = p.kv_scales[tensor - 1] + sh * p.scale_pitch + tok;
+                const float* t = p.w_table + (size_t)(tok % p.grid_w) * 2 * hw;
+                load_vec<E>(t + j0, cc);
+                load_vec<E>(t + hw + j0, ss);
             }
-            store_codes<E>(dst + lane16 * E, y, inv);
-            if (lane16 == 0) {
-                *sdst = scale;
-                if (tensor == 2) atomicMax(&s_vmax[h], __float_as_uint(scale));
+            __syncwarp();   // the previous row's reads of this slice are done
+#pragma unroll
+            for (int e = 0; e < E; e += 4) {
+                *reinterpret_cast<float4*>(cs + e) = make_float4(cc[e], cc[e + 1], cc[e + 2], cc[e + 3]);
+                *reinterpret_cast<float4*>(cs + D + e) = make_float4(ss[e], ss[e + 1], ss[e + 2], ss[e + 3]);
             }
+            __syncwarp();
         }
-    }
-    if (tensor == 2) {
-        __syncthreads();
-        for (int h = threadIdx.x; h < H; h += kThreads) {
-            const unsigned long long tag = ((unsigned long long)p.seq << 32) | s_vmax[h];
-            atomicMax(&p.v_scale_max[(size_t)p.slot[frame] * H + h], tag);
+
+        const V* item = reinterpret_cast<const V*>(src + (size_t)row * H * D + lane16 * E);
+        V raw[kItems];
+#pragma unroll
+        for (int u = 0; u < kItems; ++u) raw[u] = (row_ok && u < H) ? __ldcs(item + (size_t)u * (D / E)) : V{};
+
+        // destination of head 0 of this row, and the step from one head to the next
+        uint8_t* dst;
+        float* sdst;
+        size_t dst_step, sdst_step;
+        if (tensor == 0) {
+            dst = p.q_codes + (size_t)row * D + lane16 * E;
+            sdst = p.q_scales + row;
+            dst_step = (size_t)p.q_rows * D;
+            sdst_step = p.q_scale_pitch;
+        } else {
+            const int slot = p.ring ? p.ring->staged_slot[frame] : p.slot[frame];
+            dst = p.kv_codes[tensor - 1] + ((size_t)slot * H * T + tok) * D + lane16 * E;
+            sdst = p.kv_scales[tensor - 1] + (size_t)slot * H * p.scale_pitch + tok;
+            dst_step = (size_t)T * D;
+            sdst_step = p.scale_pitch;
+        }
+
+        for (int h0 = 0; h0 < H; h0 += kItems) {
+#pragma unroll
+            for (int u = 0; u < kItems; ++u) {
+                const int h = h0 + u;
+                const V cur = raw[u];
+                // keep kItems loads in flight: the next load of this register
+                if (row_ok && h + kItems < H) raw[u] = __ldcs(item + (size_t)(h + kItems) * (D / E));
+                float y[E];
+                unpack_bf16(cur, y);
+                if (rope) {
+                    const V praw = xor_vec(shfl_vec(cur, partner), neg_partner);
+                    float xp[E], cc[E], ss[E];
+                    unpack_bf16(praw, xp);
+#pragma unroll
+                    for (int e = 0; e < E; e += 4) {
+                        const float4 c4 = *reinterpret_cast<const float4*>(cs + e);
+                        const float4 s4 = *reinterpret_cast<const float4*>(cs + D + e);
+                        cc[e] = c4.x; cc[e + 1] = c4.y; cc[e + 2] = c4.z; cc[e + 3] = c4.w;
+                        ss[e] = s4.x; ss[e + 1] = s4.y; ss[e + 2] = s4.z; ss[e + 3] = s4.w;
+                    }
+#pragma unroll
+                    for (int e = 0; e < E; ++e)
+                        y[e] = __fadd_rn(__fmul_rn(y[e], cc[e]), __fmul_rn(xp[e], ss[e]));
+                }
+                float amax = 0.f;
+#pragma unroll
+                for (int e = 0; e < E; ++e) amax = fmaxf(amax, fabsf(y[e]));
+#pragma unroll
+                for (int o = 8; o >= 1; o >>= 1)
+                    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+                if (!row_ok || h >= H) continue;
+                const float inv = amax > 0.f ? __fdiv_rn(448.f, amax) : 0.f;
+                store_codes<E>(dst + (size_t)h * dst_step, y, inv);
+                if (lane16 == 0) {
+                    const float scale = __fdiv_rn(amax, 448.f);
+                    sdst[(size_t)h * sdst_step] = scale;
+                    if (tensor == 2) atomicMax(&s_vmax[frame][h], __float_as_uint(scale));
+                }
+            }
         }
     }
 }
 
+template <int D>
+__global__ void __launch_bounds__(kThreads, 4) append_kernel(const __grid_constant__ AppendParams p)
+{
+    __shared__ unsigned int s_vmax[kMaxFrames][kMaxHeads];   // V only: largest scale per (frame, head)
+    __shared__ __align__(16) float s_cs[kGroups * 2 * D];      // Q, K: per half-warp cos | sin of its row
+    const int tensor = blockIdx.y;             // 0 = Q, 1 = K, 2 = V
+    const int H = p.H;
+#ifdef RTV_DEBUG
+    // every staged frame must name a slot of the cache (the whole block returns alike)
+    {
+        bool bad = false;
+        for (int f = 0; f < p.n_frames; ++f) {
+            const int s = p.ring ? p.ring->staged_slot[f] : p.slot[f];
+            bad |= s < 0 || s >= p.n_slots;
+        }
+        if (bad) {
+            if (threadIdx.x == 0) atomicOr(p.err, kErrBounds);
+            return;
+        }
+    }
+#endif
+    if (tensor == 2) {
+        for (int i = threadIdx.x; i < p.n_frames * H; i += kThreads) s_vmax[i / H][i % H] = 0u;
+        __syncthreads();
+        append_rows<D, false>(p, tensor, s_vmax, s_cs);
+        __syncthreads();
+        const unsigned int seq = p.ring ? p.ring->seq : p.seq;
+        for (int i = threadIdx.x; i < p.n_frames * H; i += kThreads) {
+            const int f = i / H, h = i - f * H;
+            const int slot = p.ring ? p.ring->staged_slot[f] : p.slot[f];
+            const unsigned long long tag = ((unsigned long long)seq << 32) | s_vmax[f][h];
+            atomicMax(&p.v_scale_max[(size_t)slot * H + h], tag);
+        }
+    } else {
+        append_rows<D, true>(p, tensor, s_vmax, s_cs);
+    }
+}
+
+// Blocks per tensor: one wave of the device (resident blocks per SM x SMs,
+// shared by Q, K and V), or fewer when the chunk has fewer row groups.
+template <int D>
+cudaError_t blocks_per_tensor(int n_rows, int* out)
+{
+    static std::mutex mu;
+    static int cap[kMaxDevices] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    {
+        std::lock_guard<std::mutex> lock(mu);
+        if (!cap[dev]) {
+            int sms = 0, per_sm = 0;
+            e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+            if (e == cudaSuccess)
+                e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, append_kernel<D>, kThreads, 0);
+            if (e != cudaSuccess) return e;
+            cap[dev] = max(1, sms * max(1, per_sm) / 3);
+        }
+        *out = min(cap[dev], (n_rows + kGroups - 1) / kGroups);
+    }
+    return cudaSuccess;
+}
+
+template <int D>
+cudaError_t launch(const AppendParams& p, cudaStream_t stream)
+{
+    int bx = 0;
+    cudaError_t e = blocks_per_tensor<D>(p.n_frames * p.T, &bx);
+    if (e != cudaSuccess) return e;
+    append_kernel<D><<<dim3(bx, 3), kThreads, 0, stream>>>(p);
+    return cudaGetLastError();
+}
+
 }  // namespace
+
+cudaError_t prepare_append(int D)
+{
+    int bx = 0;
+    if (D == 128) return blocks_per_tensor<128>(1, &bx);
+    if (D == 64) return blocks_per_tensor<64>(1, &bx);
+    return cudaErrorInvalidValue;
+}
 
 cudaError_t launch_append(const AppendParams& p, int D, cudaStream_t stream)
 {
-    dim3 grid(p.n_frames * p.blocks_per_frame, 3);
-    if (D == 128)
-        append_kernel<128><<<grid, kThreads, 0, stream>>>(p);
-    else if (D == 64)
-        append_kernel<64><<<grid, kThreads, 0, stream>>>(p);
-    else
-        return cudaErrorInvalidValue;
-    return cudaGetLastError();
+    if (D == 128) return launch<128>(p, stream);
+    if (D == 64) return launch<64>(p, stream);
+    return cudaErrorInvalidValue;
 }
 
 }  // namespace rtv

@@ -35,6 +35,7 @@ struct rtv_cache {
     float* h_table = nullptr;
     float* w_table = nullptr;
     unsigned int* err = nullptr;
+    DeviceRing* dring = nullptr;        // ring state read by the kernels of a step graph
     float* part_o = nullptr;            // key-range split partials of one attention call
     int sm_count = 148;
     int last_splits = 0;
@@ -48,6 +49,7 @@ struct rtv_cache {
     unsigned int seq = 0;
     std::vector<CUtensorMap> maps;      // 5 per layer: Q, K, V, K scales, V scales
     int debug_wait_fault = 0;
+    int debug_bad_slot = -1;            // debug builds: slot the next attention names first
     long long wait_limit = 2000000000LL;
 };
 
@@ -84,7 +86,7 @@ rtv_status validate(const rtv_cache_config* c)
 
 struct Geometry {
     int T, S, q_rows, scale_pitch, q_scale_pitch;
-    size_t layer_bytes, tables_off, split_off, err_off, total;
+    size_t layer_bytes, tables_off, split_off, err_off, ring_off, total;
     rtv_layer_layout rel;   // offsets relative to the layer base
 };
 
@@ -115,7 +117,8 @@ Geometry geometry(const rtv_cache_config* c)
     const size_t split_rows = (size_t)kMaxSplit * g.q_rows * c->n_heads;
     g.split_off = align_up(g.tables_off + table_bytes, kAlign);
     g.err_off = align_up(g.split_off + split_rows * (c->head_dim + 2) * 4, kAlign);
-    g.total = align_up(g.err_off + 256, kAlign);
+    g.ring_off = align_up(g.err_off + 256, kAlign);
+    g.total = align_up(g.ring_off + sizeof(DeviceRing), kAlign);
     return g;
 }
 
@@ -218,6 +221,171 @@ int staged_slot(const rtv_cache* c, int f)
     return c->P0 + (int)((c->G + f) % c->C);
 }
 
+// Frame-axis RoPE cos/sin of absolute frame t: angle t * base^(-2j/rope_t) in fp64.
+void frame_table(const rtv_cache* c, long long t, float (*tt)[kMaxRopeHalf])
+{
+    const int half = c->cfg.rope_t / 2;
+    for (int j = 0; j < half; ++j) {
+        const double inv_freq = std::pow(c->cfg.rope_base, -2.0 * (double)j / (double)c->cfg.rope_t);
+        const double theta = (double)t * inv_freq;
+        tt[0][j] = (float)std::cos(theta);
+        tt[1][j] = (float)std::sin(theta);
+    }
+}
+
+// Launch parameters of one layer's append (no change to the cache's state).
+void fill_append_params(const rtv_cache* c, int layer, const void* q, const void* k, const void* v,
+                        int n_frames, unsigned int seq, AppendParams& p)
+{
+    const rtv_layer_layout& L = c->layout[layer];
+    std::memset(&p, 0, sizeof p);
+    p.src[0] = static_cast<const uint16_t*>(q);
+    p.src[1] = static_cast<const uint16_t*>(k);
+    p.src[2] = static_cast<const uint16_t*>(v);
+    p.q_codes = c->buf + L.q_codes;
+    p.q_scales = reinterpret_cast<float*>(c->buf + L.q_scales);
+    p.kv_codes[0] = c->buf + L.k_codes;
+    p.kv_codes[1] = c->buf + L.v_codes;
+    p.kv_scales[0] = reinterpret_cast<float*>(c->buf + L.k_scales);
+    p.kv_scales[1] = reinterpret_cast<float*>(c->buf + L.v_scales);
+    p.v_scale_max = reinterpret_cast<unsigned long long*>(c->buf + L.v_scale_max);
+    p.h_table = c->h_table;
+    p.w_table = c->w_table;
+    p.H = c->H; p.D = c->D; p.T = c->T; p.grid_w = c->cfg.grid_w; p.n_frames = n_frames;
+    p.q_rows = c->F_max * c->T;
+    p.q_scale_pitch = L.q_scale_pitch;
+    p.scale_pitch = L.scale_pitch;
+    p.n_t = c->cfg.rope_t; p.n_h = c->cfg.rope_h; p.n_w = c->cfg.rope_w;
+    p.seq = seq;
+    p.n_slots = c->S;
+    p.err = c->err;
+    const long long t0 = frames_committed(c);
+    for (int f = 0; f < n_frames; ++f) {
+        p.slot[f] = staged_slot(c, f);
+        frame_table(c, t0 + f, p.t_table[f]);
+    }
+}
+
+// Launch parameters of one layer's attention over n staged frames (no change
+// to the cache's state).  The split partials go to part_base (capacity_bytes
+// of room: n_split*M*H*D floats of O, then n_split*M*H*2 of statistics); a
+// plan whose partials do not fit is rejected with RTV_ERR_UNSUPPORTED.
+rtv_status fill_attend_params(const rtv_cache* c, int layer, void* out, int out_dtype, int n,
+                              float* part_base, size_t capacity_bytes, AttendParams& p)
+{
+    const rtv_layer_layout& L = c->layout[layer];
+    std::memset(&p, 0, sizeof p);
+    p.q_scales = reinterpret_cast<const float*>(c->buf + L.q_scales);
+    p.v_scale_max = reinterpret_cast<const unsigned long long*>(c->buf + L.v_scale_max);
+    p.out = out;
+    p.err = c->err;
+    p.H = c->H; p.D = c->D; p.T = c->T; p.M = n * c->T;
+    p.q_scale_pitch = L.q_scale_pitch;
+    p.out_bf16 = out_dtype == RTV_OUT_BF16;
+    p.tiles_per_frame = (c->T + kAttendKeys - 1) / kAttendKeys;
+    int nk = 0;
+    for (int s : c->visible_slots) p.slot[nk++] = s;
+    for (int f = 0; f < n; ++f) p.slot[nk++] = staged_slot(c, f);
+    p.n_frames_keys = nk;
+    const int units = ((p.M + 2 * kAttendRows - 1) / (2 * kAttendRows)) * p.H;
+    if (rtv_split_plan(units, nk * p.tiles_per_frame, c->sm_count, &p.n_split, &p.tiles_per_split) != RTV_OK)
+        return RTV_ERR_INVALID_ARG;
+    const size_t part_rows = (size_t)p.n_split * p.M * p.H;
+    if (p.n_split > 1 && part_rows * (p.D + 2) * sizeof(float) > capacity_bytes) return RTV_ERR_UNSUPPORTED;
+    p.part_o = part_base;
+    p.part_ml = part_base + part_rows * p.D;
+    p.n_slots = c->S;
+    p.debug_wait_fault = c->debug_wait_fault;
+    p.wait_limit = c->wait_limit;
+    return RTV_OK;
+}
+
+// Commit n staged frames to the host ring state (no device work).
+void commit_frames(rtv_cache* c, int n)
+{
+    const long long t0 = frames_committed(c);
+    for (int f = 0; f < n; ++f) {
+        const int s = staged_slot(c, f);
+        c->frame_of_slot[s] = t0 + f;
+        c->visible_frames.push_back(t0 + f);
+        c->visible_slots.push_back(s);
+    }
+    if (in_pinned_phase(c)) c->pinned_committed = true;
+    else c->G += n;
+    const size_t n_pinned = c->pinned_committed ? 1 : 0;
+    while (c->visible_frames.size() - n_pinned > (size_t)c->W) {
+        c->frame_of_slot[c->visible_slots[n_pinned]] = -1;
+        c->visible_frames.erase(c->visible_frames.begin() + n_pinned);
+        c->visible_slots.erase(c->visible_slots.begin() + n_pinned);
+    }
+    std::fill(c->staged.begin(), c->staged.end(), 0);
+}
+
+// The steady state a step graph can capture: pinned frame committed, window
+// full, nothing staged.
+bool steady(const rtv_cache* c)
+{
+    if (c->P0 && !c->pinned_committed) return false;
+    if (c->G < c->W) return false;
+    for (int n : c->staged)
+        if (n) return false;
+    return true;
+}
+
+// The device ring state of the current host state for chunks of n frames.
+void host_ring(const rtv_cache* c, int n, DeviceRing& r)
+{
+    std::memset(&r, 0, sizeof r);
+    r.G = c->G;
+    r.t0 = frames_committed(c);
+    r.seq = c->seq + 1;
+    int nk = 0;
+    for (int s : c->visible_slots) r.slot[nk++] = s;
+    for (int f = 0; f < n; ++f) {
+        r.staged_slot[f] = staged_slot(c, f);
+        r.slot[nk++] = r.staged_slot[f];
+        frame_table(c, r.t0 + f, r.t_table[f]);
+    }
+    r.n_staged = n;
+    r.P0 = c->P0;
+    r.C = c->C;
+    r.W = c->W;
+    r.n_keys = nk;
+    r.rope_half = c->cfg.rope_t / 2;
+    for (int j = 0; j < r.rope_half; ++j)
+        r.inv_freq[j] = std::pow(c->cfg.rope_base, -2.0 * (double)j / (double)c->cfg.rope_t);
+}
+
+// Advance of the device ring state by one chunk (steady state): one warp.
+// The window is generated frames G-W..G-1, the staged frames G..G+F-1, every
+// one in slot P0 + (g mod C); the frame-axis cos/sin of the new staged frames
+// use the host's fp64 inverse frequencies and the device's fp64 sincos.
+__global__ void ring_advance_kernel(DeviceRing* r)
+{
+    const int lane = threadIdx.x;
+    const int F = r->n_staged, P0 = r->P0, C = r->C, W = r->W;
+    const long long G = r->G + F;
+    const long long t0 = r->t0 + F;
+    const unsigned int seq = r->seq + 1;
+    __syncwarp();
+    for (int i = lane; i < r->n_keys; i += 32)
+        r->slot[i] = i < P0 ? 0 : P0 + (int)((G - W + (i - P0)) % C);
+    for (int f = lane; f < F; f += 32) r->staged_slot[f] = P0 + (int)((G + f) % C);
+    for (int i = lane; i < F * r->rope_half; i += 32) {
+        const int f = i / r->rope_half, j = i - f * r->rope_half;
+        double sn, cs;
+        sincos((double)(t0 + f) * r->inv_freq[j], &sn, &cs);
+        r->t_table[f][0][j] = (float)cs;
+        r->t_table[f][1][j] = (float)sn;
+    }
+    __syncwarp();
+    if (lane == 0) {
+        r->G = G;
+        r->t0 = t0;
+        r->seq = seq;
+    }
+}
+
 // Split partials of rtv_attend_static_scratch: a fixed device array (16 MiB),
 // shared by every cache and stream of the device.
 constexpr size_t kStaticScratchFloats = (size_t)4 << 20;
@@ -244,6 +412,23 @@ rtv_status static_scratch_address(int device, float** out)
 
 }  // namespace
 
+namespace rtv {
+cudaError_t launch_ring_advance(DeviceRing* ring, cudaStream_t stream)
+{
+    ring_advance_kernel<<<1, 32, 0, stream>>>(ring);
+    return cudaGetLastError();
+}
+}  // namespace rtv
+
+struct rtv_step_graph {
+    rtv_cache* cache = nullptr;
+    int n_frames = 0;
+    cudaGraph_t graph = nullptr;
+    cudaGraphExec_t exec = nullptr;
+    long long valid_G = -1;             // host state for which the device ring is current
+    unsigned int valid_seq = 0;
+};
+
 extern "C" {
 
 const char* rtv_status_string(rtv_status s)
@@ -256,6 +441,7 @@ const char* rtv_status_string(rtv_status s)
     case RTV_ERR_STATE: return "invalid state for this call";
     case RTV_ERR_TIMEOUT: return "kernel wait timed out";
     case RTV_ERR_UNSUPPORTED: return "unsupported configuration";
+    case RTV_ERR_BOUNDS: return "slot index out of range (debug build)";
     }
     return "unknown status";
 }
@@ -324,6 +510,7 @@ rtv_status rtv_cache_create(const rtv_cache_config* cfg, void* device_buf, size_
     c->h_table = reinterpret_cast<float*>(c->buf + g.tables_off);
     c->w_table = c->h_table + (size_t)cfg->grid_h * cfg->rope_h;
     c->err = reinterpret_cast<unsigned int*>(c->buf + g.err_off);
+    c->dring = reinterpret_cast<DeviceRing*>(c->buf + g.ring_off);
     c->part_o = reinterpret_cast<float*>(c->buf + g.split_off);
     {
         int sms = 0;
@@ -389,40 +576,8 @@ rtv_status rtv_cache_append(rtv_cache* c, int layer, const void* q, const void* 
         if (l != layer && c->staged[l] && c->staged[l] != n_frames) return RTV_ERR_STATE;
     if (!same_device(c)) return RTV_ERR_INVALID_ARG;
 
-    const rtv_layer_layout& L = c->layout[layer];
     AppendParams p;
-    std::memset(&p, 0, sizeof p);
-    p.src[0] = static_cast<const uint16_t*>(q);
-    p.src[1] = static_cast<const uint16_t*>(k);
-    p.src[2] = static_cast<const uint16_t*>(v);
-    p.q_codes = c->buf + L.q_codes;
-    p.q_scales = reinterpret_cast<float*>(c->buf + L.q_scales);
-    p.kv_codes[0] = c->buf + L.k_codes;
-    p.kv_codes[1] = c->buf + L.v_codes;
-    p.kv_scales[0] = reinterpret_cast<float*>(c->buf + L.k_scales);
-    p.kv_scales[1] = reinterpret_cast<float*>(c->buf + L.v_scales);
-    p.v_scale_max = reinterpret_cast<unsigned long long*>(c->buf + L.v_scale_max);
-    p.h_table = c->h_table;
-    p.w_table = c->w_table;
-    p.H = c->H; p.D = c->D; p.T = c->T; p.grid_w = c->cfg.grid_w; p.n_frames = n_frames;
-    p.rows_per_block = std::max(1, std::min(std::min(c->T, 32), 320 / c->H));
-    p.blocks_per_frame = (c->T + p.rows_per_block - 1) / p.rows_per_block;
-    p.q_rows = c->F_max * c->T;
-    p.q_scale_pitch = L.q_scale_pitch;
-    p.scale_pitch = L.scale_pitch;
-    p.n_t = c->cfg.rope_t; p.n_h = c->cfg.rope_h; p.n_w = c->cfg.rope_w;
-    p.seq = ++c->seq;
-    const long long t0 = frames_committed(c);
-    for (int f = 0; f < n_frames; ++f) {
-        p.slot[f] = staged_slot(c, f);
-        const int half = c->cfg.rope_t / 2;
-        for (int j = 0; j < half; ++j) {
-            const double inv_freq = std::pow(c->cfg.rope_base, -2.0 * (double)j / (double)c->cfg.rope_t);
-            const double theta = (double)(t0 + f) * inv_freq;
-            p.t_table[f][0][j] = (float)std::cos(theta);
-            p.t_table[f][1][j] = (float)std::sin(theta);
-        }
-    }
+    fill_append_params(c, layer, q, k, v, n_frames, ++c->seq, p);
     if (launch_append(p, c->D, static_cast<cudaStream_t>(stream)) != cudaSuccess) return RTV_ERR_CUDA;
     c->staged[layer] = n_frames;
     return RTV_OK;
@@ -467,31 +622,14 @@ rtv_status attend_impl(rtv_cache* c, int layer, void* out, int out_dtype, void* 
     if (n == 0) return RTV_ERR_STATE;
     if (!same_device(c)) return RTV_ERR_INVALID_ARG;
 
-    const rtv_layer_layout& L = c->layout[layer];
     AttendParams p;
-    std::memset(&p, 0, sizeof p);
-    p.q_scales = reinterpret_cast<const float*>(c->buf + L.q_scales);
-    p.v_scale_max = reinterpret_cast<const unsigned long long*>(c->buf + L.v_scale_max);
-    p.out = out;
-    p.err = c->err;
-    p.H = c->H; p.D = c->D; p.T = c->T; p.M = n * c->T;
-    p.q_scale_pitch = L.q_scale_pitch;
-    p.out_bf16 = out_dtype == RTV_OUT_BF16;
-    p.tiles_per_frame = (c->T + kAttendKeys - 1) / kAttendKeys;
-    int nk = 0;
-    for (int s : c->visible_slots) p.slot[nk++] = s;
-    for (int f = 0; f < n; ++f) p.slot[nk++] = staged_slot(c, f);
-    p.n_frames_keys = nk;
-    const int units = ((p.M + 2 * kAttendRows - 1) / (2 * kAttendRows)) * p.H;
-    if (rtv_split_plan(units, nk * p.tiles_per_frame, c->sm_count, &p.n_split, &p.tiles_per_split) != RTV_OK)
-        return RTV_ERR_INVALID_ARG;
-    const size_t part_rows = (size_t)p.n_split * p.M * p.H;
-    if (p.n_split > 1 && part_rows * (p.D + 2) * sizeof(float) > capacity_bytes) return RTV_ERR_UNSUPPORTED;
-    p.part_o = part_base;
-    p.part_ml = part_base + part_rows * p.D;
-    p.debug_wait_fault = c->debug_wait_fault;
-    p.wait_limit = c->wait_limit;
+    const rtv_status st = fill_attend_params(c, layer, out, out_dtype, n, part_base, capacity_bytes, p);
+    if (st != RTV_OK) return st;
     c->debug_wait_fault = 0;
+    if (c->debug_bad_slot >= 0) {
+        p.slot[0] = c->debug_bad_slot;   // only reachable in a debug build
+        c->debug_bad_slot = -1;
+    }
     c->last_splits = p.n_split;
     if (launch_attend(p, &c->maps[(size_t)layer * 5], c->D, static_cast<cudaStream_t>(stream)) !=
         cudaSuccess)
@@ -526,26 +664,11 @@ rtv_status rtv_cache_advance(rtv_cache* c)
     if (n == 0) return RTV_ERR_STATE;
     for (int l = 1; l < c->cfg.n_layers; ++l)
         if (c->staged[l] != n) return RTV_ERR_STATE;
-    const long long t0 = frames_committed(c);
     for (int f = 0; f < n; ++f) {
         const int s = staged_slot(c, f);
         if (c->frame_of_slot[s] != -1) return RTV_ERR_STATE;   // cannot happen: F <= F_max
     }
-    for (int f = 0; f < n; ++f) {
-        const int s = staged_slot(c, f);
-        c->frame_of_slot[s] = t0 + f;
-        c->visible_frames.push_back(t0 + f);
-        c->visible_slots.push_back(s);
-    }
-    if (in_pinned_phase(c)) c->pinned_committed = true;
-    else c->G += n;
-    const size_t n_pinned = c->pinned_committed ? 1 : 0;
-    while (c->visible_frames.size() - n_pinned > (size_t)c->W) {
-        c->frame_of_slot[c->visible_slots[n_pinned]] = -1;
-        c->visible_frames.erase(c->visible_frames.begin() + n_pinned);
-        c->visible_slots.erase(c->visible_slots.begin() + n_pinned);
-    }
-    std::fill(c->staged.begin(), c->staged.end(), 0);
+    commit_frames(c, n);
     return RTV_OK;
 }
 
@@ -615,6 +738,7 @@ rtv_status rtv_poll_error(rtv_cache* c)
     if (cudaDeviceSynchronize() != cudaSuccess) return RTV_ERR_CUDA;
     if (cudaMemcpy(&e, c->err, 4, cudaMemcpyDeviceToHost) != cudaSuccess) return RTV_ERR_CUDA;
     if (e && cudaMemset(c->err, 0, 4) != cudaSuccess) return RTV_ERR_CUDA;
+    if (e & kErrBounds) return RTV_ERR_BOUNDS;
     if (e & kErrTimeout) return RTV_ERR_TIMEOUT;
     return RTV_OK;
 }
@@ -625,6 +749,138 @@ rtv_status rtv_debug_set_wait_fault(rtv_cache* c, int enable, long long wait_lim
     c->debug_wait_fault = enable ? 1 : 0;
     c->wait_limit = wait_limit_cycles ? wait_limit_cycles : 2000000000LL;
     return RTV_OK;
+}
+
+int rtv_debug_build(void)
+{
+#ifdef RTV_DEBUG
+    return 1;
+#else
+    return 0;
+#endif
+}
+
+rtv_status rtv_debug_corrupt_next_attend(rtv_cache* c, int bad_slot)
+{
+    if (!c) return RTV_ERR_INVALID_ARG;
+#ifdef RTV_DEBUG
+    c->debug_bad_slot = bad_slot < 0 ? -1 : bad_slot;
+    return RTV_OK;
+#else
+    (void)bad_slot;
+    return RTV_ERR_UNSUPPORTED;
+#endif
+}
+
+rtv_status rtv_step_graph_create(rtv_cache* c, int n_frames, const void* const* q,
+                                 const void* const* k, const void* const* v, void* const* out,
+                                 int out_dtype, void* stream, rtv_step_graph** out_graph)
+{
+    if (!out_graph) return RTV_ERR_INVALID_ARG;
+    *out_graph = nullptr;
+    if (!c || !q || !k || !v || !out || !stream) return RTV_ERR_INVALID_ARG;
+    if (n_frames < 1 || n_frames > c->F_max) return RTV_ERR_INVALID_ARG;
+    if (out_dtype != RTV_OUT_F32 && out_dtype != RTV_OUT_BF16) return RTV_ERR_INVALID_ARG;
+    const int L = c->cfg.n_layers;
+    for (int l = 0; l < L; ++l)
+        if (!q[l] || !k[l] || !v[l] || !out[l] || !aligned16(q[l]) || !aligned16(k[l]) ||
+            !aligned16(v[l]) || !aligned16(out[l]))
+            return RTV_ERR_INVALID_ARG;
+    if (!same_device(c)) return RTV_ERR_INVALID_ARG;
+    if (!steady(c)) return RTV_ERR_STATE;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (prepare_append(c->D) != cudaSuccess || prepare_attend(c->D) != cudaSuccess) {
+        cudaGetLastError();
+        return RTV_ERR_CUDA;
+    }
+    DeviceRing r;
+    host_ring(c, n_frames, r);
+    std::vector<AppendParams> ap(L);
+    std::vector<AttendParams> tp(L);
+    const size_t cap = (size_t)kMaxSplit * c->F_max * c->T * c->H * (c->D + 2) * sizeof(float);
+    for (int l = 0; l < L; ++l) {
+        fill_append_params(c, l, q[l], k[l], v[l], n_frames, r.seq, ap[l]);
+        ap[l].ring = c->dring;
+        const rtv_status st = fill_attend_params(c, l, out[l], out_dtype, n_frames, c->part_o, cap, tp[l]);
+        if (st != RTV_OK) return st;
+        tp[l].ring = c->dring;
+        tp[l].debug_wait_fault = 0;
+    }
+    if (cudaMemcpyAsync(c->dring, &r, sizeof r, cudaMemcpyHostToDevice, s) != cudaSuccess ||
+        cudaStreamSynchronize(s) != cudaSuccess) {
+        cudaGetLastError();
+        return RTV_ERR_CUDA;
+    }
+    cudaGraph_t graph = nullptr;
+    if (cudaStreamBeginCapture(s, cudaStreamCaptureModeThreadLocal) != cudaSuccess) {
+        cudaGetLastError();
+        return RTV_ERR_CUDA;
+    }
+    bool ok = true;
+    for (int l = 0; l < L && ok; ++l)
+        ok = launch_append(ap[l], c->D, s) == cudaSuccess &&
+             launch_attend(tp[l], &c->maps[(size_t)l * 5], c->D, s) == cudaSuccess;
+    ok = ok && launch_ring_advance(c->dring, s) == cudaSuccess;
+    const cudaError_t e = cudaStreamEndCapture(s, &graph);
+    cudaGraphExec_t exec = nullptr;
+    if (ok && e == cudaSuccess && graph) ok = cudaGraphInstantiate(&exec, graph, 0) == cudaSuccess;
+    else ok = false;
+    rtv_step_graph* g = ok ? new (std::nothrow) rtv_step_graph() : nullptr;
+    if (!g) {
+        if (exec) cudaGraphExecDestroy(exec);
+        if (graph) cudaGraphDestroy(graph);
+        cudaGetLastError();
+        return ok ? RTV_ERR_OOM : RTV_ERR_CUDA;
+    }
+    g->cache = c;
+    g->n_frames = n_frames;
+    g->graph = graph;
+    g->exec = exec;
+    g->valid_G = c->G;
+    g->valid_seq = c->seq;
+    c->last_splits = tp[0].n_split;
+    *out_graph = g;
+    return RTV_OK;
+}
+
+rtv_status rtv_step_graph_launch(rtv_step_graph* g, void* stream)
+{
+    if (!g || !g->cache) return RTV_ERR_INVALID_ARG;
+    rtv_cache* c = g->cache;
+    if (!same_device(c)) return RTV_ERR_INVALID_ARG;
+    if (!steady(c)) return RTV_ERR_STATE;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (c->G != g->valid_G || c->seq != g->valid_seq) {
+        // direct calls moved the ring since the last replay: bring the device
+        // ring state up to date first (stream-ordered)
+        DeviceRing r;
+        host_ring(c, g->n_frames, r);
+        if (cudaMemcpyAsync(c->dring, &r, sizeof r, cudaMemcpyHostToDevice, s) != cudaSuccess) {
+            cudaGetLastError();
+            return RTV_ERR_CUDA;
+        }
+    }
+    if (cudaGraphLaunch(g->exec, s) != cudaSuccess) {
+        cudaGetLastError();
+        return RTV_ERR_CUDA;
+    }
+    // the host mirror makes the same step: every layer appended under one
+    // sequence number, then the chunk committed
+    c->seq += 1;
+    commit_frames(c, g->n_frames);
+    g->valid_G = c->G;
+    g->valid_seq = c->seq;
+    return RTV_OK;
+}
+
+rtv_status rtv_step_graph_destroy(rtv_step_graph* g)
+{
+    if (!g) return RTV_ERR_INVALID_ARG;
+    rtv_status st = RTV_OK;
+    if (g->exec && cudaGraphExecDestroy(g->exec) != cudaSuccess) st = RTV_ERR_CUDA;
+    if (g->graph && cudaGraphDestroy(g->graph) != cudaSuccess) st = RTV_ERR_CUDA;
+    delete g;
+    return st;
 }
 
 }  // extern "C"

@@ -18,12 +18,33 @@ constexpr int kMaxRopeHalf = 32;   // rope_t / 2 <= 32 (frame-axis table travels
 // Attention tiling shared by the kernel and the host-side TMA descriptors:
 // 128 query rows per query tile, 64 keys per KV tile.
 constexpr int kAttendRows = 128;
-constexpr int kAttendKeys = 64;
+constexpr int kAttendKeys = 128;
 constexpr int kMaxSplit = 4;       // key-range splits of one attention call
 constexpr int kMaxDevices = 64;    // per-device one-time set-up tables
 
 // Device error word bits.
 constexpr uint32_t kErrTimeout = 1u;
+constexpr uint32_t kErrBounds = 2u;    // debug builds: a kernel found a slot index out of range
+
+// ------------------------------------------------------ device ring state --
+// The ring state the kernels of a captured step graph read from device memory
+// (in the cache buffer), so that one graph serves every step: the host
+// uploads it when the graph is created (or when host calls moved the ring
+// since), and the advance kernel at the end of each replayed step moves it
+// one chunk forward.  Only the steady state is captured: the window is full
+// (and the pinned frame committed), so the key set has a fixed frame count.
+struct DeviceRing {
+    // moved by the advance kernel
+    long long G;                   // generated frames committed
+    long long t0;                  // absolute frame index of staged frame 0
+    unsigned int seq;              // V-scale-max tag of this step's appends
+    int slot[kMaxSlots];           // key set, logical order: pinned, window, staged
+    int staged_slot[kMaxFrames];
+    float t_table[kMaxFrames][2][kMaxRopeHalf];   // frame-axis cos/sin of the staged frames
+    // fixed for the life of a graph
+    int n_staged, P0, C, W, n_keys, rope_half;
+    double inv_freq[kMaxRopeHalf]; // rope_base^(-2j / rope_t), computed on the host
+};
 
 // ---------------------------------------------------------------- append --
 struct AppendParams {
@@ -42,8 +63,11 @@ struct AppendParams {
     int q_scale_pitch, scale_pitch;
     int n_t, n_h, n_w;
     unsigned int seq;              // append sequence number (V-scale max tag)
+    int n_slots;                   // slots of the cache (debug builds check against it)
+    unsigned int* err;             // device error word
     int slot[kMaxFrames];          // ring slot of each staged frame
     float t_table[kMaxFrames][2][kMaxRopeHalf];   // frame-axis cos/sin per staged frame
+    const DeviceRing* ring;        // non-null: take seq, slot and t_table from here
 };
 
 // ------------------------------------------------------------- attention --
@@ -61,15 +85,22 @@ struct AttendParams {
     int tiles_per_split;           // KV tiles per split (the last may hold fewer)
     float* part_o;                 // [n_split][M][H][D] unnormalised O per split
     float* part_ml;                // [n_split][M][H][2] (reference exponent, row sum)
+    int n_slots;                   // slots of the cache (debug builds check against it)
     int debug_wait_fault;          // 1: producer never arms the first barrier
     long long wait_limit;          // per-wait limit in clock cycles
     int slot[kMaxSlots];           // key set, logical order
+    const DeviceRing* ring;        // non-null: take the key set's slots from here
 };
 
 // Launchers (defined in the .cu files).
 cudaError_t launch_append(const AppendParams& p, int D, cudaStream_t stream);
 cudaError_t launch_attend(const AttendParams& p, const CUtensorMap* maps, int D,
                           cudaStream_t stream);
+cudaError_t launch_ring_advance(DeviceRing* ring, cudaStream_t stream);
+// One-time per-device launch set-up (attributes, occupancy), done before a
+// stream capture so that none of it happens inside one.
+cudaError_t prepare_append(int D);
+cudaError_t prepare_attend(int D);
 // maps: [0] Q codes, [1] K codes, [2] V codes, [3] K scales, [4] V scales
 
 }  // namespace rtv

@@ -11,7 +11,9 @@ import ctypes
 import os
 
 HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(HERE, "librtv.so")
+# RTV_LIBRARY=debug selects the bounds-checking debug build (librtv_debug.so)
+LIB_PATH = os.path.join(HERE, "librtv_debug.so" if os.environ.get("RTV_LIBRARY") == "debug"
+                        else "librtv.so")
 
 RTV_OK = 0
 RTV_ERR_INVALID_ARG = 1
@@ -20,6 +22,7 @@ RTV_ERR_CUDA = 3
 RTV_ERR_STATE = 4
 RTV_ERR_TIMEOUT = 5
 RTV_ERR_UNSUPPORTED = 6
+RTV_ERR_BOUNDS = 7
 RTV_OUT_F32 = 0
 RTV_OUT_BF16 = 1
 RTV_MAX_SLOTS = 64
@@ -73,13 +76,19 @@ _SIGS = {
     "rtv_cache_export": (_S, [_P, _S, _S, _P, _P, _P, _P, _P, _P, _P]),
     "rtv_poll_error": (_S, [_P]),
     "rtv_debug_set_wait_fault": (_S, [_P, _S, ctypes.c_longlong]),
+    "rtv_debug_build": (_S, []),
+    "rtv_debug_corrupt_next_attend": (_S, [_P, _S]),
+    "rtv_step_graph_create": (_S, [_P, _S, ctypes.POINTER(_P), ctypes.POINTER(_P), ctypes.POINTER(_P),
+                                   ctypes.POINTER(_P), _S, _P, ctypes.POINTER(_P)]),
+    "rtv_step_graph_launch": (_S, [_P, _P]),
+    "rtv_step_graph_destroy": (_S, [_P]),
 }
 
 
 def _load() -> ctypes.CDLL:
     if not os.path.exists(LIB_PATH):
-        raise ImportError(f"librtv.so not built ({LIB_PATH}); run "
-                          "`python -m kv_cache_serving_append_b200.build`")
+        raise ImportError(f"{os.path.basename(LIB_PATH)} not built ({LIB_PATH}); run "
+                          "`python -m kv_cache_serving_append_b200.build [--debug]`")
     L = ctypes.CDLL(LIB_PATH)
     for name, (res, args) in _SIGS.items():
         fn = getattr(L, name)
@@ -284,3 +293,45 @@ class Cache:
             q_scales=sl(L.q_scales, H * L.q_scale_pitch, torch.float32).view(H, L.q_scale_pitch)[:, :qr],
             v_scale_max=sl(L.v_scale_max, S * H, torch.int64).view(S, H),
         )
+
+
+class StepGraph:
+    """One captured steady-state step of every layer (append + attend each,
+    then the device-side ring advance), replayed by :meth:`launch`.  The
+    graph reads the given per-layer input tensors and writes the per-layer
+    output tensors each time it runs; they stay owned by this object."""
+
+    def __init__(self, cache: Cache, n_frames: int, qs, ks, vs, outs, stream):
+        import torch
+        L = cache.cfg["n_layers"]
+        if not all(len(x) == L for x in (qs, ks, vs, outs)):
+            raise RtvError(RTV_ERR_INVALID_ARG, "rtv_step_graph_create")
+        for t in (*qs, *ks, *vs):
+            check(cache.tensor_status(t, cache._rows(n_frames), (torch.bfloat16,)), "rtv_step_graph_create")
+        for t in outs:
+            check(cache.tensor_status(t, cache._rows(n_frames), (torch.float32, torch.bfloat16)),
+                  "rtv_step_graph_create")
+        if len({t.dtype for t in outs}) != 1:
+            raise RtvError(RTV_ERR_INVALID_ARG, "rtv_step_graph_create")
+        dt = RTV_OUT_BF16 if outs[0].dtype == torch.bfloat16 else RTV_OUT_F32
+        arr = lambda ts: (_P * L)(*[t.data_ptr() for t in ts])   # noqa: E731
+        self.cache, self.n_frames = cache, n_frames
+        self.tensors = (list(qs), list(ks), list(vs), list(outs))
+        h = _P()
+        check(lib.rtv_step_graph_create(cache.handle, n_frames, arr(qs), arr(ks), arr(vs), arr(outs), dt,
+                                        _stream_ptr(stream), ctypes.byref(h)), "rtv_step_graph_create")
+        self.handle = h
+
+    def launch(self, stream=None) -> int:
+        return lib.rtv_step_graph_launch(self.handle, _stream_ptr(stream))
+
+    def close(self):
+        if self.handle:
+            check(lib.rtv_step_graph_destroy(self.handle), "rtv_step_graph_destroy")
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass

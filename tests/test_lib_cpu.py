@@ -23,7 +23,7 @@ def rtv():
 
 def declared_symbols():
     text = open(HEADER).read()
-    return sorted(set(re.findall(r"^(?:const char\*|rtv_status)\s+(rtv_\w+)\s*\(", text, re.M)))
+    return sorted(set(re.findall(r"^(?:const char\*|rtv_status|int)\s+(rtv_\w+)\s*\(", text, re.M)))
 
 
 def test_header_declares_the_boundary():
@@ -46,7 +46,20 @@ def test_library_exports_every_declared_symbol(rtv):
     assert set(declared_symbols()) <= exported
 
 
+def test_debug_and_release_builds(rtv):
+    """librtv_debug.so (RTV_DEBUG: kernels bounds-check slot indices) exports
+    the same symbols and says it is the debug build; the release library
+    refuses the debug-only test hook."""
+    from kv_cache_serving_append_b200 import build
+    dbg = ctypes.CDLL(build.build(debug=True))
+    assert dbg.rtv_debug_build() == 1
+    assert rtv.lib.rtv_debug_build() == 0
+    assert not [s for s in declared_symbols() if not hasattr(dbg, s)]
+    assert rtv.lib.rtv_debug_corrupt_next_attend(None, 3) == rtv.RTV_ERR_INVALID_ARG
+
+
 def test_status_strings(rtv):
+    assert rtv.status_string(7) == "slot index out of range (debug build)"
     for s in range(7):
         assert rtv.status_string(s)
     assert rtv.status_string(5) == "kernel wait timed out"
@@ -120,15 +133,15 @@ def test_injected_allocation_failure_returns_oom():
 
 def test_split_plan_choices_and_invariants(rtv):
     """The key-range split rtv_attend uses (host arithmetic, no device)."""
-    # full-shape layer, ring full: 12 row blocks x 40 heads, 9 frames x 47 tiles, 148 SMs:
-    # 480 CTAs = 3.24 waves unsplit; 4 splits of <= 106 tiles -> 13 waves of quarter CTAs
-    assert rtv.split_plan(480, 9 * 47, 148) == (4, 106)
-    # the same layer's first step (one frame of keys): still 4 splits, of 12 tiles (last 11)
-    assert rtv.split_plan(480, 47, 148) == (4, 12)
-    # two frames per chunk, W=16 + pinned: 24 x 40 units, 19 x 47 tiles -> 2 splits
-    assert rtv.split_plan(960, 19 * 47, 148) == (2, 447)
-    # 704-token frames, 8 heads, 7 frames of 11 tiles: 24 units fill a fraction of the GPU
-    assert rtv.split_plan(24, 77, 148) == (4, 20)
+    # full-shape layer, ring full: 12 row blocks x 40 heads, 9 frames x 24 tiles of 128 keys,
+    # 148 SMs: 480 CTAs = 3.24 waves unsplit; 4 splits of 54 tiles -> 13 waves of quarter CTAs
+    assert rtv.split_plan(480, 9 * 24, 148) == (4, 54)
+    # the same layer's first step (one frame of keys): 24 tiles allow 3 splits of 8
+    assert rtv.split_plan(480, 24, 148) == (3, 8)
+    # two frames per chunk, W=16 + pinned: 24 x 40 units, 19 x 24 tiles -> 2 splits
+    assert rtv.split_plan(960, 19 * 24, 148) == (2, 228)
+    # 704-token frames, 8 heads, 7 frames of 6 tiles: 24 units fill a fraction of the GPU
+    assert rtv.split_plan(24, 42, 148) == (4, 11)
     # too few tiles to split (fewer than 8 per split)
     assert rtv.split_plan(2, 5, 148) == (1, 5)
     assert rtv.split_plan(480, 15, 148) == (1, 15)
