@@ -519,6 +519,71 @@ def time_e2e(res, steps: int, warmup: int, world: int, dev):
     return ms / steps, h2d_bytes, d2h_bytes
 
 
+def time_project(dev, steps: int, warmup: int) -> dict:
+    """The fused QKV projection + append (rtv_cache_append_project) at the
+    full layer shape: a 2992 x 15360 x 5120 FP8 GEMM whose epilogue writes
+    the cache.  For context, the path it replaces: three library FP8 GEMMs
+    (torch._scaled_mm, one per Q/K/V, bf16 out) and then rtv_cache_append."""
+    import torch
+    from kv_cache_serving_append_b200 import configs, rtv, synth
+    cfg = configs.get(CFG_ID)
+    hidden = 5120
+    H, D = cfg["n_heads"], cfg["head_dim"]
+    T = cfg["grid_h"] * cfg["grid_w"]
+    HD = H * D
+    cache = rtv.Cache(cfg, dev)
+    xc, sx, wc, sw = (torch.from_numpy(a).to(dev) for a in synth.projection_inputs(cfg, 0, 0, 1, hidden, False))
+    stream = torch.cuda.current_stream(dev)
+
+    def fused():
+        if cache.append_project(0, xc, sx, wc, sw, 1, stream):
+            raise RuntimeError("append_project failed")
+
+    def timed(fn, n):
+        for _ in range(warmup):
+            fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(n):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / n
+
+    flop = 2.0 * T * 3 * HD * hidden
+    res = {"workload": "QKV projection (FP8 GEMM 2992 x 15360 x 5120, per-row / per-feature scales) "
+                       "with the append fused into its epilogue, full layer shape",
+           "gemm_flop": flop}
+    fused_ms = timed(fused, steps)
+    res["fused_us"] = fused_ms * 1e3
+    res["fused_tflops"] = flop / (fused_ms * 1e-3) / 1e12
+    if cache.poll_error():
+        raise RuntimeError("kernel error in the fused projection")
+    try:
+        x8 = xc.view(torch.float8_e4m3fn)
+        w8 = [wc[i * HD:(i + 1) * HD].view(torch.float8_e4m3fn) for i in range(3)]
+        ws = [sw[i * HD:(i + 1) * HD].view(1, HD) for i in range(3)]
+        xs = sx.view(T, 1)
+        outs = [torch.empty((T, HD), dtype=torch.bfloat16, device=dev) for _ in range(3)]
+
+        def unfused():
+            for i in range(3):
+                torch._scaled_mm(x8, w8[i].t(), scale_a=xs, scale_b=ws[i], out_dtype=torch.bfloat16,
+                                 out=outs[i])
+            if cache.append(0, outs[0].view(T, H, D), outs[1].view(T, H, D), outs[2].view(T, H, D), 1, stream):
+                raise RuntimeError("append failed")
+
+        un_ms = timed(unfused, steps)
+        res["unfused_us"] = un_ms * 1e3
+        res["unfused_path"] = "3 x torch._scaled_mm (rowwise scales, bf16 out) + rtv_cache_append"
+    except Exception as e:   # the library GEMM is context only
+        res["unfused_us"] = None
+        res["unfused_error"] = str(e)[:200]
+    cache.close()
+    return res
+
+
 def extra_workloads(dev, steps: int, warmup: int):
     """The other full-shape workloads, each timed on its own (one GPU)."""
     import torch
@@ -550,6 +615,7 @@ def extra_workloads(dev, steps: int, warmup: int):
     torch.cuda.empty_cache()
     out["seq48_graph"] = run_seq48_graph_timing(dev, min(steps, 5), 2)
     torch.cuda.empty_cache()
+    out["project_append"] = time_project(dev, k, 3)
     return out
 
 

@@ -198,6 +198,33 @@ rtv_status rtv_cache_append(rtv_cache* cache, int layer, const void* q, const vo
                             const void* v, int n_frames, void* stream);
 
 /*
+ * The QKV projection with the append fused into it: an FP8 GEMM on tcgen05
+ * tensor cores whose epilogue does rtv_cache_append's work on the projected
+ * Q/K/V, so the bf16 Q/K/V are never written to or read from memory.
+ * Source: lhc.media, "Runway partage la construction de Runway Characters",
+ * third paragraph (matmul and kernel tuning); aidose.in, "Runway explains how
+ * it serves a 57B video model in real time", third paragraph (FP8 matmuls;
+ * rotary embedding and FP8 quantisation applied once, at cache write).
+ *   x_codes   E4M3 [n_frames*T][hidden] activations, row-major, 16-byte aligned
+ *   x_scales  fp32 [n_frames*T], one per token row
+ *   w_codes   E4M3 [3*n_heads*head_dim][hidden] weights, row-major (one output
+ *             feature per row: the Q heads, then the K heads, then the V
+ *             heads, each head's head_dim features contiguous), 16-byte aligned
+ *   w_scales  fp32 [3*n_heads*head_dim], one per output feature, 16-byte aligned
+ *   hidden    a multiple of 128
+ * The projected value of row r, feature n is
+ *     bf16( fl( fl(acc * x_scales[r]) * w_scales[n] ) ),
+ *     acc = sum_k decode(x_codes[r][k]) * decode(w_codes[n][k]) (fp32),
+ * and the cache then receives exactly what rtv_cache_append would write for
+ * that bf16 Q/K/V (same staging, overwrite and frame rules).  Supported for
+ * head_dim 128 with the RoPE split 32:48:48 and an even n_heads.
+ * Errors: as rtv_cache_append, plus RTV_ERR_UNSUPPORTED (other shapes).
+ */
+rtv_status rtv_cache_append_project(rtv_cache* cache, int layer, const void* x_codes,
+                                    const float* x_scales, const void* w_codes,
+                                    const float* w_scales, int hidden, int n_frames, void* stream);
+
+/*
  * Attention of the layer's staged chunk over its key set (pinned frame,
  * window oldest to newest, staged frames).
  * Source: aidose.in, "Runway explains how it serves a 57B video model in real

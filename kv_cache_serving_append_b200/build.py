@@ -17,7 +17,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "librtv.so")
 LIB_DEBUG = os.path.join(HERE, "librtv_debug.so")   # RTV_DEBUG: kernels bounds-check slot indices
-SOURCES = ["rtv_cache.cu", "append_kernel.cu", "attend_kernel.cu"]
+SOURCES = ["rtv_cache.cu", "append_kernel.cu", "attend_kernel.cu", "project_kernel.cu"]
 HEADERS = ["rtv_internal.h", "sm100.cuh", os.path.join("..", "..", "include", "rtv.h")]
 
 NVCC_FLAGS = [

@@ -583,6 +583,61 @@ rtv_status rtv_cache_append(rtv_cache* c, int layer, const void* q, const void* 
     return RTV_OK;
 }
 
+rtv_status rtv_cache_append_project(rtv_cache* c, int layer, const void* x_codes, const float* x_scales,
+                                    const void* w_codes, const float* w_scales, int hidden, int n_frames,
+                                    void* stream)
+{
+    if (!c || layer < 0 || layer >= c->cfg.n_layers) return RTV_ERR_INVALID_ARG;
+    if (!x_codes || !x_scales || !w_codes || !w_scales || !aligned16(x_codes) || !aligned16(w_codes) ||
+        !aligned16(w_scales) || ((uintptr_t)x_scales & 3))
+        return RTV_ERR_INVALID_ARG;
+    if (hidden < 128 || hidden % 128) return RTV_ERR_INVALID_ARG;
+    if (n_frames < 1 || n_frames > c->F_max) return RTV_ERR_INVALID_ARG;
+    if (in_pinned_phase(c) && n_frames != 1) return RTV_ERR_INVALID_ARG;
+    // the fused epilogue is specialised to the workloads' head shape
+    if (c->D != 128 || c->cfg.rope_t != 32 || c->cfg.rope_h != 48 || c->cfg.rope_w != 48 || (c->H % 2))
+        return RTV_ERR_UNSUPPORTED;
+    for (int l = 0; l < c->cfg.n_layers; ++l)
+        if (l != layer && c->staged[l] && c->staged[l] != n_frames) return RTV_ERR_STATE;
+    if (!same_device(c)) return RTV_ERR_INVALID_ARG;
+    const int rows = n_frames * c->T;
+    const int feats = 3 * c->H * c->D;
+    CUtensorMap maps[2];
+    {
+        cuuint64_t dims[2] = {(cuuint64_t)hidden, (cuuint64_t)rows};
+        cuuint64_t st[1] = {(cuuint64_t)hidden};
+        cuuint32_t box[2] = {128, 128};
+        if (!encode(&maps[0], CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(x_codes), dims, st, box,
+                    CU_TENSOR_MAP_SWIZZLE_128B))
+            return RTV_ERR_CUDA;
+    }
+    {
+        cuuint64_t dims[2] = {(cuuint64_t)hidden, (cuuint64_t)feats};
+        cuuint64_t st[1] = {(cuuint64_t)hidden};
+        cuuint32_t box[2] = {128, 256};
+        if (!encode(&maps[1], CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(w_codes), dims, st, box,
+                    CU_TENSOR_MAP_SWIZZLE_128B))
+            return RTV_ERR_CUDA;
+    }
+    ProjectParams p;
+    std::memset(&p, 0, sizeof p);
+    fill_append_params(c, layer, nullptr, nullptr, nullptr, n_frames, ++c->seq, p.a);
+    p.sx = x_scales;
+    p.sw = w_scales;
+    p.R = rows;
+    p.Kd = hidden;
+    p.n_m_tiles = (rows + 127) / 128;
+    p.n_n_tiles = feats / 256;
+    p.wait_limit = c->wait_limit;
+    p.err = c->err;
+    if (launch_project(p, maps, c->sm_count, static_cast<cudaStream_t>(stream)) != cudaSuccess) {
+        cudaGetLastError();
+        return RTV_ERR_CUDA;
+    }
+    c->staged[layer] = n_frames;
+    return RTV_OK;
+}
+
 rtv_status rtv_split_plan(int n_units, int n_kv_tiles, int sm_count, int* n_split, int* tiles_per_split)
 {
     if (n_units < 1 || n_kv_tiles < 1 || sm_count < 1 || !n_split || !tiles_per_split)

@@ -92,6 +92,20 @@ struct AttendParams {
     const DeviceRing* ring;        // non-null: take the key set's slots from here
 };
 
+// ----------------------------------------------- projection + append --
+// x codes [R][Kd] E4M3 with s_x [R]; w codes [3*H*D][Kd] E4M3 with s_w [3*H*D]
+// (rows: Q heads, then K heads, then V heads, each head's D features
+// contiguous); the append part as for rtv_cache_append.
+struct ProjectParams {
+    AppendParams a;
+    const float* sx;
+    const float* sw;
+    int R, Kd;
+    int n_m_tiles, n_n_tiles;      // ceil(R / 128), 3*H*D / 256
+    long long wait_limit;
+    unsigned int* err;
+};
+
 // Launchers (defined in the .cu files).
 cudaError_t launch_append(const AppendParams& p, int D, cudaStream_t stream);
 cudaError_t launch_attend(const AttendParams& p, const CUtensorMap* maps, int D,
@@ -101,6 +115,9 @@ cudaError_t launch_ring_advance(DeviceRing* ring, cudaStream_t stream);
 // stream capture so that none of it happens inside one.
 cudaError_t prepare_append(int D);
 cudaError_t prepare_attend(int D);
+cudaError_t prepare_project();
+cudaError_t launch_project(const ProjectParams& p, const CUtensorMap* maps, int sm_count,
+                           cudaStream_t stream);
 // maps: [0] Q codes, [1] K codes, [2] V codes, [3] K scales, [4] V scales
 
 }  // namespace rtv

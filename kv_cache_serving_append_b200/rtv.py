@@ -68,6 +68,7 @@ _SIGS = {
     "rtv_cache_destroy": (_S, [_P]),
     "rtv_cache_append": (_S, [_P, _S, _P, _P, _P, _S, _P]),
     "rtv_attend": (_S, [_P, _S, _P, _S, _P]),
+    "rtv_cache_append_project": (_S, [_P, _S, _P, _P, _P, _P, _S, _S, _P]),
     "rtv_attend_static_scratch": (_S, [_P, _S, _P, _S, _P]),
     "rtv_split_plan": (_S, [_S, _S, _S, ctypes.POINTER(_S), ctypes.POINTER(_S)]),
     "rtv_cache_advance": (_S, [_P]),
@@ -213,6 +214,29 @@ class Cache:
                 return st
         st = lib.rtv_cache_append(self.handle, layer, _ptr(q), _ptr(k), _ptr(v), n_frames,
                                   _stream_ptr(stream))
+        if st == RTV_OK:
+            self._staged[layer] = n_frames
+        return st
+
+    def append_project(self, layer: int, x_codes, x_scales, w_codes, w_scales, n_frames: int,
+                       stream=None) -> int:
+        """Fused QKV projection (FP8 GEMM) + append: x_codes uint8 [n_frames*T, hidden],
+        x_scales fp32 [n_frames*T], w_codes uint8 [3*H*D, hidden], w_scales fp32 [3*H*D]."""
+        import torch
+        if not isinstance(n_frames, int) or not 1 <= n_frames <= self.cfg["max_frames_per_chunk"]:
+            return RTV_ERR_INVALID_ARG
+        rows = n_frames * self.T
+        feats = 3 * self.cfg["n_heads"] * self.cfg["head_dim"]
+        if getattr(x_codes, "dim", lambda: 0)() != 2 or x_codes.shape[0] != rows:
+            return RTV_ERR_INVALID_ARG
+        hidden = x_codes.shape[1]
+        for t, n, dt in ((x_codes, rows * hidden, torch.uint8), (x_scales, rows, torch.float32),
+                         (w_codes, feats * hidden, torch.uint8), (w_scales, feats, torch.float32)):
+            st = self.tensor_status(t, n, (dt,))
+            if st != RTV_OK:
+                return st
+        st = lib.rtv_cache_append_project(self.handle, layer, _ptr(x_codes), _ptr(x_scales), _ptr(w_codes),
+                                          _ptr(w_scales), hidden, n_frames, _stream_ptr(stream))
         if st == RTV_OK:
             self._staged[layer] = n_frames
         return st

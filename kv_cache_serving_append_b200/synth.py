@@ -82,3 +82,33 @@ def chunk(cfg_id, cfg: dict, layer: int, step: int, n_frames: int, device="cpu",
 def bf16_bits(x: torch.Tensor):
     """bf16 tensor -> numpy uint16 bit patterns (host copy)."""
     return x.detach().cpu().contiguous().view(torch.int16).numpy().view("uint16")
+
+
+def projection_inputs(cfg: dict, layer: int, step: int, n_frames: int, hidden: int, exact: bool,
+                      seed_offset: int = 0):
+    """E4M3 codes and fp32 scales for the fused projection: activations
+    x [n_frames*T, hidden] with one scale per row, weights w [3*H*D, hidden]
+    with one scale per output feature.  ``exact``: codes only from the binades
+    [0.5, 1) and [1, 2) (random sign, some zeros), whose products are
+    multiples of 2^-8 below 4, so any fp32 sum of up to 2^14 of them is exact
+    whatever the order; otherwise codes of a N(0, 1) draw.  Returns numpy
+    (x_codes, x_scales, w_codes, w_scales)."""
+    import numpy as np
+    T = cfg["grid_h"] * cfg["grid_w"]
+    rows, feats = n_frames * T, 3 * cfg["n_heads"] * cfg["head_dim"]
+    rng = np.random.default_rng(7 * (seed_of(2, layer, step) + 1) + 3 * hidden + seed_offset)
+
+    def codes(shape):
+        if exact:
+            c = ((rng.integers(6, 8, shape) << 3) | rng.integers(0, 8, shape)).astype(np.uint8)
+            c |= (rng.integers(0, 2, shape) << 7).astype(np.uint8)
+            c[rng.random(shape) < 0.02] = 0
+            return c
+        import torch
+        x = torch.from_numpy(rng.standard_normal(shape).astype(np.float32) * 64.0)
+        return x.clamp(-448, 448).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+
+    xc, wc = codes((rows, hidden)), codes((feats, hidden))
+    sx = (rng.uniform(0.5, 2.0, rows) / 64.0).astype(np.float32)
+    sw = (rng.uniform(0.5, 2.0, feats) / (64.0 * np.sqrt(hidden))).astype(np.float32)
+    return xc, sx, wc, sw

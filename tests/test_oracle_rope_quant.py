@@ -148,3 +148,39 @@ def test_append_tensor_v_unrotated_and_positions():
         rot = oracle.rope3d(xf[:, h], SPLITS[D], pos)
         c3, s3, _ = oracle.quantize_rows(rot)
         assert np.array_equal(kc[h], c3) and np.array_equal(ks[h], s3)
+
+
+def test_bf16_rounding_matches_torch():
+    """The oracle's fp32 -> bf16 rounding against PyTorch's cast (an
+    independent implementation of round-to-nearest-even), including ties."""
+    import torch
+    rng = np.random.default_rng(11)
+    v = rng.standard_normal(200000).astype(np.float32) * np.float32(3.0)
+    u = v.view(np.uint32)
+    ties = ((u & 0xFFFF0000) | 0x8000).view(np.float32)            # exactly halfway
+    both = np.concatenate([v, ties, np.float32([0.0, -0.0, 1.0, 65504.0, 1e-38])])
+    ref = torch.from_numpy(both).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(oracle.bf16_rne_bits(both), ref)
+
+
+def test_projection_definition_on_a_brute_force_case():
+    """project_qkv against a per-element loop over the definition (decode,
+    products summed in fp64, two fp32 scale multiplies, bf16 rounding)."""
+    rng = np.random.default_rng(12)
+    xc = rng.integers(0, 256, (5, 16)).astype(np.uint8)
+    wc = rng.integers(0, 256, (7, 16)).astype(np.uint8)
+    for c in (xc, wc):
+        c[(c & 0x7F) == 0x7F] = 0x40
+    sx = rng.uniform(0.1, 1, 5).astype(np.float32)
+    sw = rng.uniform(0.1, 1, 7).astype(np.float32)
+    got = oracle.project_qkv(xc, sx, wc, sw)
+    dx, dw = oracle.e4m3_decode(xc), oracle.e4m3_decode(wc)
+    for r in range(5):
+        for n in range(7):
+            acc = 0.0
+            for k in range(16):
+                acc += dx[r, k] * dw[n, k]
+            v = np.float32(np.float32(np.float32(acc) * sx[r]) * sw[n])
+            import torch
+            ref = torch.tensor([float(v)], dtype=torch.float32).to(torch.bfloat16).view(torch.int16).item() & 0xFFFF
+            assert got[r, n] == ref, (r, n)
