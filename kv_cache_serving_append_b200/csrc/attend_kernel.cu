@@ -77,7 +77,7 @@ constexpr uint32_t kTmemCols = 512;
 // polynomial on the FMA pipe instead of the MUFU ex2 unit (0: none), which
 // runs short of throughput before the tensor pipe does.
 #ifndef RTV_POLY_EVERY
-#define RTV_POLY_EVERY 4
+#define RTV_POLY_EVERY 0
 #endif
 constexpr int kPolyEvery = RTV_POLY_EVERY;
 constexpr int kLazyRescaleLog2 = 8;     // move the reference when a tile's row sum reaches 2^8 of it
