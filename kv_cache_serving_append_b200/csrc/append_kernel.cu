@@ -77,32 +77,6 @@ __device__ __forceinline__ uint2 shfl_vec(const uint2& v, int src)
 __device__ __forceinline__ uint4 xor_vec(const uint4& v, uint32_t m) { return make_uint4(v.x ^ m, v.y ^ m, v.z ^ m, v.w ^ m); }
 __device__ __forceinline__ uint2 xor_vec(const uint2& v, uint32_t m) { return make_uint2(v.x ^ m, v.y ^ m); }
 
-// Packed fp32 pairs (sm_100 f32x2 arithmetic): one instruction, two
-// independent IEEE round-to-nearest operations, so results are those of the
-// scalar forms bit for bit.
-__device__ __forceinline__ uint64_t pack2(float a, float b)
-{
-    uint64_t r;
-    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
-    return r;
-}
-__device__ __forceinline__ void unpack2(uint64_t r, float& a, float& b)
-{
-    asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(r));
-}
-__device__ __forceinline__ uint64_t mul2(uint64_t a, uint64_t b)
-{
-    uint64_t r;
-    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
-    return r;
-}
-__device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b)
-{
-    uint64_t r;
-    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
-    return r;
-}
-
 // E4M3 round-to-nearest-even with saturation to +-448 (hardware cvt).
 __device__ __forceinline__ uint16_t e4m3x2(float lo, float hi)
 {
@@ -114,12 +88,10 @@ __device__ __forceinline__ void store_codes(uint8_t* dst, const float* y, float 
 template <>
 __device__ __forceinline__ void store_codes<8>(uint8_t* dst, const float* y, float inv)
 {
-    const uint64_t ii = pack2(inv, inv);
-    float q[8];
-#pragma unroll
-    for (int e = 0; e < 8; e += 2) unpack2(mul2(pack2(y[e], y[e + 1]), ii), q[e], q[e + 1]);
-    uint32_t w0 = e4m3x2(q[0], q[1]) | ((uint32_t)e4m3x2(q[2], q[3]) << 16);
-    uint32_t w1 = e4m3x2(q[4], q[5]) | ((uint32_t)e4m3x2(q[6], q[7]) << 16);
+    uint32_t w0 = e4m3x2(__fmul_rn(y[0], inv), __fmul_rn(y[1], inv)) |
+                  ((uint32_t)e4m3x2(__fmul_rn(y[2], inv), __fmul_rn(y[3], inv)) << 16);
+    uint32_t w1 = e4m3x2(__fmul_rn(y[4], inv), __fmul_rn(y[5], inv)) |
+                  ((uint32_t)e4m3x2(__fmul_rn(y[6], inv), __fmul_rn(y[7], inv)) << 16);
     *reinterpret_cast<uint2*>(dst) = make_uint2(w0, w1);
 }
 template <>
@@ -259,12 +231,9 @@ __device__ __forceinline__ void append_rows(const AppendParams& p, int tensor,
                         cc[e] = c4.x; cc[e + 1] = c4.y; cc[e + 2] = c4.z; cc[e + 3] = c4.w;
                         ss[e] = s4.x; ss[e + 1] = s4.y; ss[e + 2] = s4.z; ss[e + 3] = s4.w;
                     }
-                    // y = fl(x c) + fl(x_partner s) per element, two elements per instruction
 #pragma unroll
-                    for (int e = 0; e < E; e += 2)
-                        unpack2(add2(mul2(pack2(y[e], y[e + 1]), pack2(cc[e], cc[e + 1])),
-                                     mul2(pack2(xp[e], xp[e + 1]), pack2(ss[e], ss[e + 1]))),
-                                y[e], y[e + 1]);
+                    for (int e = 0; e < E; ++e)
+                        y[e] = __fadd_rn(__fmul_rn(y[e], cc[e]), __fmul_rn(xp[e], ss[e]));
                 }
                 float amax = 0.f;
 #pragma unroll

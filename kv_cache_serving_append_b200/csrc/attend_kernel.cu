@@ -16,8 +16,7 @@
 //   warp 0     TMA producer: both Q tiles once; per KV tile the K and V code
 //              tiles at (ring slot * H + head, token tile) and their scales.
 //   warp 1     MMA issuer for both query tiles (and TMEM owner):
-//                QK_0(0) QK_1(0) | QKa_0(j+1) PV_0(j) QKb_0(j+1) |
-//                QKa_1(j+1) PV_1(j) QKb_1(j+1) | ...
+//                QK_0(0) QK_1(0) | PV_0(j) QK_0(j+1) | PV_1(j) QK_1(j+1) | ...
 //              S_t = Q_t K_j^T is kind::f8f6f4 (E4M3 x E4M3 -> f32 in TMEM);
 //              O_t += P_t V16_j is kind::f16 with P read from TMEM, where the
 //              softmax wrote it over S_t, and V16 from shared memory.  While
@@ -34,15 +33,9 @@
 //              sum reaches 2^15 (f16 P range), and m moves up by a power of
 //              two, with O rescaled lazily, only when a row sum reaches 2^8.
 // TMEM columns: S_0 [0,128), S_1 [128,256), O_0 [256,256+D), O_1 [384,384+D).
-// Each S_t is two 64-column regions; a tile's scores for keys [0, 64) (half A)
-// go to region A(j) = 64 * (j & 1) and keys [64, 128) (half B) to the other
-// region, and its P (128 keys of f16 = 64 columns) is written over region
-// A(j), whose scores are already in registers by then.  So QK_t(j+1)'s half A
-// (region A(j+1), which held tile j's half B, consumed) is issued right after
-// softmax t released tile j, ahead of PV_t(j), and the next softmax starts on
-// it while PV_t(j) and QK_t(j+1)'s half B run; half B overwrites region A(j)
-// behind PV_t(j), which reads P out of it -- tcgen05 MMAs from one issuing
-// thread execute in order, so the write cannot overtake the read.
+// QK_t(j+1) overwrites S_t right after PV_t(j), which reads P_t out of it,
+// is issued: tcgen05 MMAs from one issuing thread execute in order, so the
+// write cannot overtake the read.
 //
 // Logical-to-physical frame order is resolved in the TMA coordinates: the
 // kernel receives the key set as a list of ring slots -- no gather, no copy.
@@ -107,8 +100,7 @@ struct Smem {
     uint64_t q_full;
     uint64_t k_full[kStages];       // K, V codes and scales of a stage landed
     uint64_t kv_empty[kStages];     // every reader of a stage is done with it
-    uint64_t s_full_a[kQT];         // QK_t(j) over keys [0, 64) complete
-    uint64_t s_full_b[kQT];         // QK_t(j) over keys [64, 128) complete (tiles with more than 64 keys)
+    uint64_t s_full[kQT];           // QK_t(j) complete
     uint64_t p_ready[kQT];          // softmax t wrote P_t(j)
     uint64_t pv_done[kQT];          // PV_t(j) complete
     uint64_t v16_ready[kNV16];      // V16 buffer widened
@@ -258,18 +250,17 @@ __device__ __forceinline__ float tile_row_max(const uint32_t* sr, const float* s
     return fmaxf(fmaxf(mt[0], mt[1]), fmaxf(mt[2], mt[3]));
 }
 
-// One pass over chunks [c0, c1) of a KV tile (32 keys each; the scores of this
-// thread's row in registers): u = s * scale_k, x = u*c2 + neg (= (u - m)*c2 -
-// log2 Sv for the reference m), p/Sv = 2^x, P = (p/Sv) * scale_v packed to f16
-// pairs and written to TMEM at t_s (keys [32c, 32c+32) -> P columns
-// [16c, 16c+16), columns whose scores are already in registers).  Only the ceil(nv/32) chunks that hold valid keys are done (the
+// One pass over a KV tile (the scores of this thread's row in registers):
+// u = s * scale_k, x = u*c2 + neg (= (u - m)*c2 - log2 Sv for the reference
+// m), p/Sv = 2^x, P = (p/Sv) * scale_v packed to f16 pairs and written over S
+// in TMEM (keys [32c, 32c+32) -> P columns [16c, 16c+16); S is already in
+// registers).  Only the ceil(nv/32) chunks that hold valid keys are done (the
 // PV MMA reads P for ceil(nv/16)*16 keys), and only a chunk that holds the
 // tile's last valid key masks (warp-uniform branch).  Returns the row sum of
 // p/Sv, which also bounds every p/Sv of the tile: the caller reads from it
 // whether the tile outgrew m.
 __device__ __forceinline__ float tile_exp(const uint32_t* sr, uint32_t t_s, const float* sk,
-                                          const float* sv, uint64_t c2c2, uint64_t neg2, int nv,
-                                          int c0, int c1)
+                                          const float* sv, uint64_t c2c2, uint64_t neg2, int nv)
 {
     const float4* sk4 = reinterpret_cast<const float4*>(sk);
     const float4* sv4 = reinterpret_cast<const float4*>(sv);
@@ -277,7 +268,6 @@ __device__ __forceinline__ float tile_exp(const uint32_t* sr, uint32_t t_s, cons
     uint64_t ls2[4] = {pack2(0.f, 0.f), pack2(0.f, 0.f), pack2(0.f, 0.f), pack2(0.f, 0.f)};
 #pragma unroll
     for (int c = 0; c < kBN / 32; ++c) {
-        if (c < c0 || c >= c1) continue;
         if (32 * c >= nv) break;
         const bool mask = 32 * c + 32 > nv;
         uint32_t pk[16];
@@ -368,8 +358,7 @@ attend_kernel(const __grid_constant__ AttendParams p, const __grid_constant__ CU
             mbar_init(&sm.kv_empty[s], 1 + 2 + 4 * n_qt);
         }
         for (int t = 0; t < kQT; ++t) {
-            mbar_init(&sm.s_full_a[t], 1);
-            mbar_init(&sm.s_full_b[t], 1);
+            mbar_init(&sm.s_full[t], 1);
             mbar_init(&sm.p_ready[t], 4);
             mbar_init(&sm.pv_done[t], 1);
         }
@@ -439,55 +428,62 @@ attend_kernel(const __grid_constant__ AttendParams p, const __grid_constant__ CU
                 constexpr uint32_t kSw = D == 128 ? kSwizzle128 : kSwizzle64;
                 constexpr uint32_t kSbo = D == 128 ? 1024 : 512;
                 constexpr uint32_t kPV = idesc(kBM, D, 0, 0, 0, 1);          // f16 x f16(MN) -> f32
-                // S_t = Q_t K_j^T for keys [64*half, 64*half + 64) of the tile (N =
-                // its valid keys rounded up to 16) into the half's region
-                auto issue_qk = [&](int t, int j, int half) -> bool {
-                    const int nh = min(64, tile_at(p, j0 + j).nv - 64 * half);
-                    if (nh <= 0) return true;
+                constexpr uint32_t kKVBytes = Smem<D>::kKVBytes, kV16Bytes = Smem<D>::kV16Bytes;
+                // Descriptors are computed once: a buffer or K step only moves the
+                // start-address field (bits 0-13, address >> 4; shared memory is
+                // below 256 KB, so the add never carries out of the field).
+                const uint64_t q_desc[kQT] = {smem_desc(smem_u32(sm.q[0]), 16, kSbo, kSw),
+                                              smem_desc(smem_u32(sm.q[1]), 16, kSbo, kSw)};
+                const uint64_t k_desc0 = smem_desc(smem_u32(sm.k[0]), 16, kSbo, kSw);
+                const uint64_t v_desc0 = smem_desc(smem_u32(sm.v16[0]), kBN * 128, 1024, kSwizzle128);
+                const uint32_t qk_full = idesc(kBM, kBN, 0, 0, 0, 0);        // E4M3 x E4M3 -> f32
+                // valid keys of each tile, walked without divisions
+                int fr = j0 % p.tiles_per_frame;                             // tile within its frame
+                int nv_next = min(kBN, p.T - fr * kBN);                      // keys of the next QK tile
+                int nv_cur = 0;                                              // keys of the tile PV works on
+                auto step_tile = [&]() {
+                    nv_cur = nv_next;
+                    if (++fr == p.tiles_per_frame) fr = 0;
+                    nv_next = min(kBN, p.T - fr * kBN);
+                };
+                // S_t = Q_t K_j^T over N = the tile's valid keys rounded up to 16
+                auto issue_qk = [&](int t, int j, int nv) -> bool {
                     if (!mbar_wait(&sm.k_full[j % kStages], (j / kStages) & 1, limit)) return false;
                     tc_fence_after();
-                    const uint32_t n16 = (uint32_t)((nh + 15) & ~15);
-                    const uint32_t qk = idesc(kBM, n16, 0, 0, 0, 0);          // E4M3 x E4M3 -> f32
-                    const uint32_t q_addr = smem_u32(sm.q[t]);
-                    const uint32_t k_addr = smem_u32(sm.k[j % kStages]) + 64 * half * D;
-                    const uint32_t region = (64u * ((j & 1) ^ half));
+                    const uint32_t qk = nv == kBN ? qk_full : idesc(kBM, (uint32_t)((nv + 15) & ~15), 0, 0, 0, 0);
+                    const uint64_t kd = k_desc0 + (uint64_t)(((j % kStages) * kKVBytes) >> 4);
 #pragma unroll
                     for (int kk = 0; kk < D / 32; ++kk)
-                        mma_f8_ss(tmem + col_s(t) + region, smem_desc(q_addr + kk * 32, 16, kSbo, kSw),
-                                  smem_desc(k_addr + kk * 32, 16, kSbo, kSw), qk, kk > 0);
-                    tc_commit(half ? &sm.s_full_b[t] : &sm.s_full_a[t]);
+                        mma_f8_ss(tmem + col_s(t), q_desc[t] + (uint64_t)(kk * 2), kd + (uint64_t)(kk * 2), qk, kk > 0);
+                    tc_commit(&sm.s_full[t]);
                     return true;
                 };
-                // O_t += P_t V16_j over K = the tile's valid keys rounded up to 16;
-                // P_t sits in region A(j) of S_t
-                auto issue_pv = [&](int t, int j) -> bool {
+                // O_t += P_t V16_j over K = the tile's valid keys rounded up to 16
+                auto issue_pv = [&](int t, int j, int nv) -> bool {
+                    if (!mbar_wait(&sm.p_ready[t], j & 1, limit)) return false;
                     if (!mbar_wait(&sm.v16_ready[j % kNV16], (j / kNV16) & 1, limit)) return false;
                     tc_fence_after();
-                    const int nv = tile_at(p, j0 + j).nv;
-                    const uint32_t v_addr = smem_u32(sm.v16[j % kNV16]);
-                    const uint32_t pcol = col_s(t) + 64u * (j & 1);
-                    for (int kk = 0; kk < (nv + 15) / 16; ++kk)
-                        mma_f16_ts(tmem + col_o(t), tmem + pcol + kk * 8,
-                                   smem_desc(v_addr + kk * 2048, kBN * 128, 1024, kSwizzle128), kPV,
+                    const uint64_t vd = v_desc0 + (uint64_t)(((j % kNV16) * kV16Bytes) >> 4);
+                    const int n16 = (nv + 15) / 16;
+                    for (int kk = 0; kk < n16; ++kk)
+                        mma_f16_ts(tmem + col_o(t), tmem + col_s(t) + kk * 8, vd + (uint64_t)(kk * 128), kPV,
                                    (j > 0 || kk > 0) ? 1u : 0u);
                     tc_commit(&sm.pv_done[t]);
                     return true;
                 };
                 if (!mbar_wait(&sm.q_full, 0, limit)) fail = true;
+                step_tile();                                                 // nv_cur = tile 0
                 for (int t = 0; t < n_qt && !fail; ++t)
-                    if (!issue_qk(t, 0, 0) || !issue_qk(t, 0, 1)) fail = true;
+                    if (!issue_qk(t, 0, nv_cur)) fail = true;
                 if (!fail) tc_commit(&sm.kv_empty[0]);
                 for (int j = 0; j < n_tiles && !fail; ++j) {
+                    const int nv_pv = nv_cur;
+                    if (j + 1 < n_tiles) step_tile();                        // nv_cur = tile j + 1
                     for (int t = 0; t < n_qt; ++t) {
-                        if (!mbar_wait(&sm.p_ready[t], j & 1, limit)) { fail = true; break; }
-                        tc_fence_after();
-                        // half A of the next tile goes to the region tile j's half B
-                        // used (already read), ahead of PV_t(j)
-                        if (j + 1 < n_tiles && !issue_qk(t, j + 1, 0)) { fail = true; break; }
-                        if (!issue_pv(t, j)) { fail = true; break; }
-                        // half B overwrites P_t(j)'s region right behind PV_t(j):
-                        // MMAs from one thread execute in issue order
-                        if (j + 1 < n_tiles && !issue_qk(t, j + 1, 1)) { fail = true; break; }
+                        if (!issue_pv(t, j, nv_pv)) { fail = true; break; }
+                        // S_t is rewritten right behind PV_t(j), which reads P_t out of
+                        // it: MMAs from one thread execute in issue order
+                        if (j + 1 < n_tiles && !issue_qk(t, j + 1, nv_cur)) { fail = true; break; }
                     }
                     if (fail) break;
                     tc_commit(&sm.v16_free[j % kNV16]);
@@ -577,55 +573,32 @@ attend_kernel(const __grid_constant__ AttendParams p, const __grid_constant__ CU
             float o_scale = 1.f;   // factor O still owes (applied before the next PV)
             const uint64_t c2c2 = pack2(c2, c2);
             const int log2_sv_i = ve - 127;
-            int nb = 0;            // half-B completions waited for so far
             for (int j = 0; j < n_tiles && !fail; ++j) {
                 const int st = j % kStages;
                 const int nv = tile_at(p, j0 + j).nv;
-                const bool has_b = nv > 64;
-                const uint32_t t_a = t_s + 64u * (j & 1);           // half A scores, then P
-                const uint32_t t_b = t_s + 64u * ((j & 1) ^ 1);     // half B scores
                 if (!warp_wait(&sm.k_full[st], (j / kStages) & 1, limit)) { fail = true; break; }
-                if (!warp_wait(&sm.s_full_a[t], j & 1, limit)) { fail = true; break; }
+                if (!warp_wait(&sm.s_full[t], j & 1, limit)) { fail = true; break; }
                 tc_fence_after();
                 uint32_t sr[kBN];
 #pragma unroll
-                for (int c = 0; c < 2; ++c)
-                    if (32 * c < nv) tmem_ld32(t_a + c * 32, sr + c * 32);
-                // the first tile sets the reference from its exact max: both halves first
-                bool b_loaded = false;
-                if (j == 0 && has_b) {
-                    if (!warp_wait(&sm.s_full_b[t], nb & 1, limit)) { fail = true; break; }
-                    ++nb;
-                    tc_fence_after();
-#pragma unroll
-                    for (int c = 2; c < 4; ++c)
-                        if (32 * c < nv) tmem_ld32(t_b + (c - 2) * 32, sr + c * 32);
-                    b_loaded = true;
-                }
+                for (int c = 0; c < kBN / 32; ++c)
+                    if (32 * c < nv) tmem_ld32(t_s + c * 32, sr + c * 32);
                 tc_wait_ld();
-                if (j == 0) m = tile_row_max(sr, sm.sk[st], nv);
-                // single pass against the reference: p/Sv = 2^(u*c2 - m*c2 - log2 Sv),
-                // half A while half B is still being computed.  The row sum
-                // bounds every p of the tile; if some row's sum (times Sv) reaches
-                // 2^15, a p may be past f16 P range and the tile is redone once
-                // against its exact max (rare: the first tiles of a row).
-                // ls_e = floor(log2(row sum * Sv)).
-                float neg = -(m * c2 + log2_sv);
-                float ls = tile_exp(sr, t_a, sm.sk[st], sm.sv[st], c2c2, pack2(neg, neg), nv, 0, 2);
-                if (has_b) {
-                    if (!b_loaded) {
-                        if (!warp_wait(&sm.s_full_b[t], nb & 1, limit)) { fail = true; break; }
-                        ++nb;
-                        tc_fence_after();
-#pragma unroll
-                        for (int c = 2; c < 4; ++c)
-                            if (32 * c < nv) tmem_ld32(t_b + (c - 2) * 32, sr + c * 32);
-                        tc_wait_ld();
-                    }
-                    ls += tile_exp(sr, t_a, sm.sk[st], sm.sv[st], c2c2, pack2(neg, neg), nv, 2, 4);
-                }
-                int ls_e = (int)((__float_as_uint(ls) >> 23) & 0xff) - 127 + log2_sv_i;
-                if (__any_sync(0xffffffffu, ls_e >= kRedoLog2)) {
+                if (j == 0)   // the first tile sets the reference
+                    m = tile_row_max(sr, sm.sk[st], nv);
+                // single pass against the reference: p/Sv = 2^(u*c2 - m*c2 - log2 Sv).
+                // The row sum bounds every p of the tile; if some row's sum
+                // (times Sv) reaches 2^15, a p may be past f16 P range and the
+                // pass is redone once against the tile's exact max (rare: the
+                // first tiles of a row).  ls_e = floor(log2(row sum * Sv)).
+                float ls = 0.f;
+                int ls_e = 0;
+#pragma unroll 1
+                for (int attempt = 0; attempt < 2; ++attempt) {
+                    const float neg = -(m * c2 + log2_sv);
+                    ls = tile_exp(sr, t_s, sm.sk[st], sm.sv[st], c2c2, pack2(neg, neg), nv);
+                    ls_e = (int)((__float_as_uint(ls) >> 23) & 0xff) - 127 + log2_sv_i;
+                    if (attempt == 1 || !__any_sync(0xffffffffu, ls_e >= kRedoLog2)) break;
                     const float mt = tile_row_max(sr, sm.sk[st], nv);
                     const float m_new = fmaxf(m, mt);
                     const float alpha = ex2((m - m_new) * c2);
@@ -633,9 +606,6 @@ attend_kernel(const __grid_constant__ AttendParams p, const __grid_constant__ CU
                     o_scale *= alpha;
                     m = m_new;
                     tc_wait_st();   // the first pass's P stores land before they are overwritten
-                    neg = -(m * c2 + log2_sv);
-                    ls = tile_exp(sr, t_a, sm.sk[st], sm.sv[st], c2c2, pack2(neg, neg), nv, 0, 4);
-                    ls_e = (int)((__float_as_uint(ls) >> 23) & 0xff) - 127 + log2_sv_i;
                 }
                 l += ls;
                 // O owes a factor from an earlier move of m: apply it once PV(j-1)
