@@ -335,7 +335,7 @@ rtv_status rtv_poll_error(rtv_cache* cache);
 /*
  * The key-range split rtv_attend chooses (host arithmetic only; no device
  * needed).  n_units = ceil(n_frames*T / 256) * n_heads CTAs of one key range
- * each, n_kv_tiles = key frames * ceil(T / 128), sm_count = the device's SMs.
+ * each, n_kv_tiles = key frames * ceil(T / 64), sm_count = the device's SMs.
  * Out: n_split in 1..4 and tiles_per_split (the last split may hold fewer,
  * none is empty).  The plan minimises ceil(n_units*s / sm_count) / s plus 3%
  * per extra split, with at least 8 KV tiles per split.

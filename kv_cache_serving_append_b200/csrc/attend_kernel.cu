@@ -9,33 +9,31 @@
 // (pinned frame, window, chunk) and the 1/sqrt(D) softmax are the library's
 // definition, stated in rtv.h.
 //
-// One CTA = two 128-row query tiles of one head and one range of the key set,
-// sharing every K/V tile it loads.  KV tiles hold 128 keys of one frame (the
-// last tile of a frame holds T mod 128 keys and runs its MMAs with N and K
-// rounded up to 16 only).  12 warps:
+// One CTA = two 128-row query tiles of one head, sharing every K/V tile it
+// loads; KV tiles of 64 keys; 12 warps:
 //   warp 0     TMA producer: both Q tiles once; per KV tile the K and V code
 //              tiles at (ring slot * H + head, token tile) and their scales.
-//   warp 1     MMA issuer for both query tiles (and TMEM owner):
-//                QK_0(0) QK_1(0) | PV_0(j) QK_0(j+1) | PV_1(j) QK_1(j+1) | ...
-//              S_t = Q_t K_j^T is kind::f8f6f4 (E4M3 x E4M3 -> f32 in TMEM);
-//              O_t += P_t V16_j is kind::f16 with P read from TMEM, where the
-//              softmax wrote it over S_t, and V16 from shared memory.  While
-//              softmax t works on tile j, the tensor pipe runs the other query
-//              tile's PV and next QK.
-//   warps 2,3  widen the V code tile to f16 (exact), 64 keys each, in the
-//              MN-major layout the PV MMA reads.
+//   warps 1,3  MMA issuers, one per query tile t (warp 1 also owns TMEM).
+//              S_t,b = Q_t K_j^T (kind::f8f6f4, E4M3 x E4M3 -> f32 in TMEM,
+//              b = j mod 2: two S buffers per query tile), O_t += P_t,b V16_j
+//              (kind::f16, P read from TMEM where it overwrote S_t,b, V16
+//              from shared memory).  With two S buffers the softmax of KV tile
+//              j+1 runs while PV(j) and QK(j+2) execute.
+//   warp 2     widens the V code tile to f16 (exact) in the MN-major layout
+//              the PV MMA reads.
 //   warps 4-7  softmax of query tile 0, warps 8-11 of query tile 1; one query
-//              row per thread, the tile's 128 scores in registers, one pass
+//              row per thread, the tile's 64 scores in registers, one pass
 //              per KV tile against a reference m: s*scale_k, exp2, row sum,
 //              P = p*scale_v/Sv in f16 written back over S.  The row sum
 //              bounds every p of the tile, so it alone decides (no per-key
 //              max): a tile is redone against its exact max only when a row
 //              sum reaches 2^15 (f16 P range), and m moves up by a power of
 //              two, with O rescaled lazily, only when a row sum reaches 2^8.
-// TMEM columns: S_0 [0,128), S_1 [128,256), O_0 [256,256+D), O_1 [384,384+D).
-// QK_t(j+1) overwrites S_t right after PV_t(j), which reads P_t out of it,
-// is issued: tcgen05 MMAs from one issuing thread execute in order, so the
-// write cannot overtake the read.
+//              The two warpgroups run concurrently.
+// TMEM columns: S_t,b at 64*(2t+b) (64 columns each), O_0 [256,256+D),
+// O_1 [384,384+D).  QK(j+2) overwrites S_t,b right after PV(j), which reads
+// P_t,b out of it, is issued: tcgen05 MMAs from one issuing thread execute in
+// order, so the write cannot overtake the read.
 //
 // Logical-to-physical frame order is resolved in the TMA coordinates: the
 // kernel receives the key set as a list of ring slots -- no gather, no copy.
@@ -66,24 +64,17 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kBM = kAttendRows;   // query rows per query tile (128)
+constexpr int kBM = kAttendRows;   // query rows per query tile
 constexpr int kQT = 2;             // query tiles per CTA
-constexpr int kBN = kAttendKeys;   // keys per KV tile (128)
-constexpr int kStages = 3;         // K/V code tile stages
-constexpr int kNV16 = 2;           // f16 V tile buffers
+constexpr int kBN = kAttendKeys;   // keys per KV tile
+constexpr int kStages = 6;         // K/V code tile stages
+constexpr int kNV16 = 4;           // f16 V tile buffers
 constexpr int kThreads = 384;
 constexpr uint32_t kTmemCols = 512;
-// Every kPolyEvery-th score pair of a 32-key chunk takes its exp2 from a
-// polynomial on the FMA pipe instead of the MUFU ex2 unit (0: none), which
-// runs short of throughput before the tensor pipe does.
-#ifndef RTV_POLY_EVERY
-#define RTV_POLY_EVERY 0
-#endif
-constexpr int kPolyEvery = RTV_POLY_EVERY;
 constexpr int kLazyRescaleLog2 = 8;     // move the reference when a tile's row sum reaches 2^8 of it
 constexpr int kRedoLog2 = 15;           // redo a tile whose row sum reaches 2^15 (f16 P range)
 
-__host__ __device__ constexpr uint32_t col_s(int t) { return 128u * t; }
+__host__ __device__ constexpr uint32_t col_s(int t, int b) { return 64u * (2 * t + b); }
 __host__ __device__ constexpr uint32_t col_o(int t) { return 256u + 128u * t; }
 
 template <int D>
@@ -98,14 +89,11 @@ struct Smem {
     alignas(128) float sk[kStages][kBN];
     alignas(128) float sv[kStages][kBN];
     uint64_t q_full;
-    uint64_t k_full[kStages];       // K, V codes and scales of a stage landed
-    uint64_t kv_empty[kStages];     // every reader of a stage is done with it
-    uint64_t s_full[kQT];           // QK_t(j) complete
-    uint64_t p_ready[kQT];          // softmax t wrote P_t(j)
-    uint64_t pv_done[kQT];          // PV_t(j) complete
-    uint64_t v16_ready[kNV16];      // V16 buffer widened
-    uint64_t v16_free[kNV16];       // every PV that read a V16 buffer completed
-    uint64_t drain;
+    uint64_t k_full[kStages];
+    uint64_t kv_empty[kStages];
+    uint64_t s_full[kQT][2], p_ready[kQT][2], pv_done[kQT][2];
+    uint64_t v16_ready[kNV16], tile_done[kNV16];
+    uint64_t drain[kQT];
     uint32_t tmem_base;
 };
 
@@ -151,36 +139,6 @@ __device__ __forceinline__ float max3(float a, float b, float c)
     asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
     return r;
 }
-// 2^x for a pair of arguments on the FMA pipe (Cody-Waite range reduction
-// x = n + f, n = rint(x), f in [-1/2, 1/2], then a degree-4 polynomial for 2^f
-// and n added to the exponent field).  The coefficients are a minimax fit of
-// the relative error of 2^f on [-1/2, 1/2] with p(0) = 1 (Remez exchange;
-// max relative error 5.4e-6, far below the f16 rounding of P).  x is clamped
-// to [-125, 126] so the exponent stays in range: 2^-125 stands for anything
-// smaller (negligible beside a row sum of at least 2^-60) and 2^126 for
-// anything larger (the row sum then reaches the redo threshold).
-__device__ __forceinline__ uint64_t exp2_poly2(float x0, float x1)
-{
-    x0 = fminf(fmaxf(x0, -125.f), 126.f);
-    x1 = fminf(fmaxf(x1, -125.f), 126.f);
-    const uint64_t magic = pack2(12582912.f, 12582912.f);       // 1.5 * 2^23
-    const uint64_t x = pack2(x0, x1);
-    const uint64_t j = add2(x, magic);                          // rint(x) in the low mantissa bits
-    const uint64_t n = add2(j, pack2(-12582912.f, -12582912.f));
-    float n0, n1;
-    unpack2(n, n0, n1);
-    const uint64_t f = add2(x, pack2(-n0, -n1));
-    uint64_t q = fma2(pack2(9.676037356e-03f, 9.676037356e-03f), f, pack2(5.600578710e-02f, 5.600578710e-02f));
-    q = fma2(q, f, pack2(2.402216792e-01f, 2.402216792e-01f));
-    q = fma2(q, f, pack2(6.931053400e-01f, 6.931053400e-01f));
-    q = fma2(q, f, pack2(1.f, 1.f));
-    float q0, q1, j0, j1;
-    unpack2(q, q0, q1);
-    unpack2(j, j0, j1);
-    return pack2(__int_as_float(__float_as_int(q0) + (__float_as_int(j0) << 23)),
-                 __int_as_float(__float_as_int(q1) + (__float_as_int(j1) << 23)));
-}
-
 // Four E4M3 codes (bytes of w) -> four f16 (exact), as two packed pairs.
 __device__ __forceinline__ void e4m3x4_to_f16x4(uint32_t w, uint32_t& lo, uint32_t& hi)
 {
@@ -188,6 +146,13 @@ __device__ __forceinline__ void e4m3x4_to_f16x4(uint32_t w, uint32_t& lo, uint32
         "cvt.rn.f16x2.e4m3x2 %0, a;\n\tcvt.rn.f16x2.e4m3x2 %1, b;\n\t}"
         : "=r"(lo), "=r"(hi)
         : "r"(w));
+}
+
+// Ring slot of frame f of the key set (from the device ring state when the
+// launch belongs to a captured step graph).
+__device__ __forceinline__ int key_slot(const AttendParams& p, int f)
+{
+    return p.ring ? p.ring->slot[f] : p.slot[f];
 }
 
 // Bounded wait whose outcome is the same for every lane of the warp, so that
@@ -201,30 +166,10 @@ __device__ __forceinline__ bool warp_wait_sleep(uint64_t* bar, uint32_t parity, 
     return __all_sync(0xffffffffu, mbar_wait_sleep(bar, parity, limit));
 }
 
-// Ring slot of frame f of the key set (from the device ring state when the
-// launch belongs to a captured step graph).
-__device__ __forceinline__ int key_slot(const AttendParams& p, int f)
-{
-    return p.ring ? p.ring->slot[f] : p.slot[f];
-}
-
-// Where KV tile jg of the key set lives: key frame fi (an index into the
-// launch's slot list) and first token t0; nv valid keys.
-struct TileAt {
-    int fi, t0, nv;
-};
-__device__ __forceinline__ TileAt tile_at(const AttendParams& p, int jg)
-{
-    TileAt r;
-    r.fi = jg / p.tiles_per_frame;
-    r.t0 = (jg - r.fi * p.tiles_per_frame) * kBN;
-    r.nv = min(kBN, p.T - r.t0);
-    return r;
-}
-
-// Row max of u = s * scale_k over the valid keys of a KV tile (the tile's
-// scores of this thread's row are in registers).  Used for the first KV tile
-// and when a tile's scores outgrow the reference by more than f16 P allows.
+// Row max of u = s * scale_k over the valid keys of a KV tile (the kBN scores
+// of this thread's row are in registers).  Used for the first KV tile and
+// when a tile's scores outgrow the running max by more than f16 P allows.
+template <bool kMask>
 __device__ __forceinline__ float tile_row_max(const uint32_t* sr, const float* sk, int nv)
 {
     const float4* sk4 = reinterpret_cast<const float4*>(sk);
@@ -237,28 +182,29 @@ __device__ __forceinline__ float tile_row_max(const uint32_t* sr, const float* s
                      pack2(kk.x, kk.y)), a, b);
         unpack2(mul2(pack2(__uint_as_float(sr[4 * k4 + 2]), __uint_as_float(sr[4 * k4 + 3])),
                      pack2(kk.z, kk.w)), c, d);
-        const int k = 4 * k4;
-        if (k + 4 <= nv) {
-            mt[(k4 & 1) * 2] = max3(mt[(k4 & 1) * 2], a, b);
-            mt[(k4 & 1) * 2 + 1] = max3(mt[(k4 & 1) * 2 + 1], c, d);
+        float& m0 = mt[(k4 & 1) * 2];
+        float& m1 = mt[(k4 & 1) * 2 + 1];
+        if (!kMask) {
+            m0 = max3(m0, a, b);
+            m1 = max3(m1, c, d);
         } else {
-            if (k < nv) mt[0] = fmaxf(mt[0], a);
-            if (k + 1 < nv) mt[1] = fmaxf(mt[1], b);
-            if (k + 2 < nv) mt[2] = fmaxf(mt[2], c);
+            const int k = 4 * k4;
+            if (k < nv) m0 = fmaxf(m0, a);
+            if (k + 1 < nv) m1 = fmaxf(m1, b);
+            if (k + 2 < nv) m0 = fmaxf(m0, c);
+            if (k + 3 < nv) m1 = fmaxf(m1, d);
         }
     }
     return fmaxf(fmaxf(mt[0], mt[1]), fmaxf(mt[2], mt[3]));
 }
 
-// One pass over a KV tile (the scores of this thread's row in registers):
+// One pass over a KV tile (the kBN scores of this thread's row in registers):
 // u = s * scale_k, x = u*c2 + neg (= (u - m)*c2 - log2 Sv for the reference
 // m), p/Sv = 2^x, P = (p/Sv) * scale_v packed to f16 pairs and written over S
 // in TMEM (keys [32c, 32c+32) -> P columns [16c, 16c+16); S is already in
-// registers).  Only the ceil(nv/32) chunks that hold valid keys are done (the
-// PV MMA reads P for ceil(nv/16)*16 keys), and only a chunk that holds the
-// tile's last valid key masks (warp-uniform branch).  Returns the row sum of
-// p/Sv, which also bounds every p/Sv of the tile: the caller reads from it
-// whether the tile outgrew m.
+// registers).  Returns the row sum of p/Sv, which also bounds every p/Sv of
+// the tile: the caller reads from it whether the tile outgrew m.
+template <bool kMask>
 __device__ __forceinline__ float tile_exp(const uint32_t* sr, uint32_t t_s, const float* sk,
                                           const float* sv, uint64_t c2c2, uint64_t neg2, int nv)
 {
@@ -268,8 +214,6 @@ __device__ __forceinline__ float tile_exp(const uint32_t* sr, uint32_t t_s, cons
     uint64_t ls2[4] = {pack2(0.f, 0.f), pack2(0.f, 0.f), pack2(0.f, 0.f), pack2(0.f, 0.f)};
 #pragma unroll
     for (int c = 0; c < kBN / 32; ++c) {
-        if (32 * c >= nv) break;
-        const bool mask = 32 * c + 32 > nv;
         uint32_t pk[16];
 #pragma unroll
         for (int k4 = 0; k4 < 8; ++k4) {
@@ -282,17 +226,12 @@ __device__ __forceinline__ float tile_exp(const uint32_t* sr, uint32_t t_s, cons
                                         hh ? pack2(kk.z, kk.w) : pack2(kk.x, kk.y));
                 float x0, x1;
                 unpack2(fma2(u, c2c2, neg2), x0, x1);
-                if (mask) {
+                if (kMask) {
                     if (k >= nv) x0 = -INFINITY;
                     if (k + 1 >= nv) x1 = -INFINITY;
                 }
-                uint64_t pp;
-                const int pair = 2 * k4 + hh;
-                if (kPolyEvery > 0 && pair % (kPolyEvery > 0 ? kPolyEvery : 1) == kPolyEvery - 1 && !mask) {
-                    pp = exp2_poly2(x0, x1);
-                } else {
-                    pp = pack2(ex2(x0), ex2(x1));   // ex2(-inf) = 0 for masked keys
-                }
+                const float p0 = ex2(x0), p1 = ex2(x1);   // ex2(-inf) = 0 for masked keys
+                const uint64_t pp = pack2(p0, p1);
                 ls2[(k >> 1) & 3] = add2(ls2[(k >> 1) & 3], pp);
                 float q0, q1;
                 unpack2(mul2(pp, hh ? pack2(vv.z, vv.w) : pack2(vv.x, vv.y)), q0, q1);
@@ -351,22 +290,23 @@ attend_kernel(const __grid_constant__ AttendParams p, const __grid_constant__ CU
 
     if (threadIdx.x == 0) {
         mbar_init(&sm.q_full, 1);
-        // a stage is free once the QK MMAs (one commit), both widening warps and
-        // every softmax warp of an active query tile are done with it
+        // kv_empty / tile_done: one commit from each active query tile's issuer
         for (int s = 0; s < kStages; ++s) {
             mbar_init(&sm.k_full[s], 1);
-            mbar_init(&sm.kv_empty[s], 1 + 2 + 4 * n_qt);
+            mbar_init(&sm.kv_empty[s], n_qt);
         }
         for (int t = 0; t < kQT; ++t) {
-            mbar_init(&sm.s_full[t], 1);
-            mbar_init(&sm.p_ready[t], 4);
-            mbar_init(&sm.pv_done[t], 1);
+            for (int b = 0; b < 2; ++b) {
+                mbar_init(&sm.s_full[t][b], 1);
+                mbar_init(&sm.p_ready[t][b], 128);
+                mbar_init(&sm.pv_done[t][b], 1);
+            }
+            mbar_init(&sm.drain[t], 1);
         }
         for (int b = 0; b < kNV16; ++b) {
-            mbar_init(&sm.v16_ready[b], 2);
-            mbar_init(&sm.v16_free[b], 1);
+            mbar_init(&sm.v16_ready[b], 32);
+            mbar_init(&sm.tile_done[b], n_qt);
         }
-        mbar_init(&sm.drain, 1);
         fence_mbar_init();
     }
     if (warp == 1) {
@@ -405,14 +345,14 @@ attend_kernel(const __grid_constant__ AttendParams p, const __grid_constant__ CU
                         fail = true;
                         break;
                     }
-                    const TileAt ta = tile_at(p, j0 + j);
-                    const int row = key_slot(p, ta.fi) * H + h;
-                    // full boxes: rows past the frame's last token are zero-filled and counted
+                    const int fi = (j0 + j) / p.tiles_per_frame;
+                    const int t0 = (j0 + j - fi * p.tiles_per_frame) * kBN;
+                    const int row = key_slot(p, fi) * H + h;
                     mbar_arrive_expect_tx(&sm.k_full[st], 2 * kKVBytes + 2 * kBN * 4);
-                    tma_load_3d(sm.k[st], &map_k, &sm.k_full[st], 0, ta.t0, row);
-                    tma_load_3d(sm.v8[st], &map_v, &sm.k_full[st], 0, ta.t0, row);
-                    tma_load_2d(sm.sk[st], &map_sk, &sm.k_full[st], ta.t0, row);
-                    tma_load_2d(sm.sv[st], &map_sv, &sm.k_full[st], ta.t0, row);
+                    tma_load_3d(sm.k[st], &map_k, &sm.k_full[st], 0, t0, row);
+                    tma_load_3d(sm.v8[st], &map_v, &sm.k_full[st], 0, t0, row);
+                    tma_load_2d(sm.sk[st], &map_sk, &sm.k_full[st], t0, row);
+                    tma_load_2d(sm.sv[st], &map_sv, &sm.k_full[st], t0, row);
                     ++issued;
                 }
                 // drain: every copy this thread issued has landed before the CTA may exit
@@ -422,100 +362,77 @@ attend_kernel(const __grid_constant__ AttendParams p, const __grid_constant__ CU
                     mbar_wait(&sm.k_full[j % kStages], (j / kStages) & 1, limit);
                 }
             }
-        } else if (warp == 1) {
-            // ------------------------------------------------- MMA issuer --
-            if (lane == 0) {
+        } else if (warp == 1 || warp == 3) {
+            // ------------------------------------- MMA issuer of query tile t --
+            const int t = warp == 1 ? 0 : 1;
+            if (lane == 0 && t < n_qt) {
+                constexpr uint32_t kQK = idesc(kBM, kBN, 0, 0, 0, 0);        // E4M3 x E4M3 -> f32
+                constexpr uint32_t kPV = idesc(kBM, D, 0, 0, 0, 1);          // f16 x f16(MN) -> f32
                 constexpr uint32_t kSw = D == 128 ? kSwizzle128 : kSwizzle64;
                 constexpr uint32_t kSbo = D == 128 ? 1024 : 512;
-                constexpr uint32_t kPV = idesc(kBM, D, 0, 0, 0, 1);          // f16 x f16(MN) -> f32
                 constexpr uint32_t kKVBytes = Smem<D>::kKVBytes, kV16Bytes = Smem<D>::kV16Bytes;
                 // Descriptors are computed once: a buffer or K step only moves the
                 // start-address field (bits 0-13, address >> 4; shared memory is
                 // below 256 KB, so the add never carries out of the field).
-                const uint64_t q_desc[kQT] = {smem_desc(smem_u32(sm.q[0]), 16, kSbo, kSw),
-                                              smem_desc(smem_u32(sm.q[1]), 16, kSbo, kSw)};
+                const uint64_t q_desc = smem_desc(smem_u32(sm.q[t]), 16, kSbo, kSw);
                 const uint64_t k_desc0 = smem_desc(smem_u32(sm.k[0]), 16, kSbo, kSw);
                 const uint64_t v_desc0 = smem_desc(smem_u32(sm.v16[0]), kBN * 128, 1024, kSwizzle128);
-                const uint32_t qk_full = idesc(kBM, kBN, 0, 0, 0, 0);        // E4M3 x E4M3 -> f32
-                // valid keys of each tile, walked without divisions
-                int fr = j0 % p.tiles_per_frame;                             // tile within its frame
-                int nv_next = min(kBN, p.T - fr * kBN);                      // keys of the next QK tile
-                int nv_cur = 0;                                              // keys of the tile PV works on
-                auto step_tile = [&]() {
-                    nv_cur = nv_next;
-                    if (++fr == p.tiles_per_frame) fr = 0;
-                    nv_next = min(kBN, p.T - fr * kBN);
-                };
-                // S_t = Q_t K_j^T over N = the tile's valid keys rounded up to 16
-                auto issue_qk = [&](int t, int j, int nv) -> bool {
-                    if (!mbar_wait(&sm.k_full[j % kStages], (j / kStages) & 1, limit)) return false;
+                // S_t,b = Q_t K_j^T, b = j & 1, once K_j has landed
+                auto issue_qk = [&](int j) -> bool {
+                    if (!mbar_wait_backoff(&sm.k_full[j % kStages], (j / kStages) & 1, limit)) return false;
                     tc_fence_after();
-                    const uint32_t qk = nv == kBN ? qk_full : idesc(kBM, (uint32_t)((nv + 15) & ~15), 0, 0, 0, 0);
                     const uint64_t kd = k_desc0 + (uint64_t)(((j % kStages) * kKVBytes) >> 4);
 #pragma unroll
                     for (int kk = 0; kk < D / 32; ++kk)
-                        mma_f8_ss(tmem + col_s(t), q_desc[t] + (uint64_t)(kk * 2), kd + (uint64_t)(kk * 2), qk, kk > 0);
-                    tc_commit(&sm.s_full[t]);
+                        mma_f8_ss(tmem + col_s(t, j & 1), q_desc + (uint64_t)(kk * 2), kd + (uint64_t)(kk * 2),
+                                  kQK, kk > 0);
+                    tc_commit(&sm.s_full[t][j & 1]);
                     return true;
                 };
-                // O_t += P_t V16_j over K = the tile's valid keys rounded up to 16
-                auto issue_pv = [&](int t, int j, int nv) -> bool {
-                    if (!mbar_wait(&sm.p_ready[t], j & 1, limit)) return false;
-                    if (!mbar_wait(&sm.v16_ready[j % kNV16], (j / kNV16) & 1, limit)) return false;
-                    tc_fence_after();
-                    const uint64_t vd = v_desc0 + (uint64_t)(((j % kNV16) * kV16Bytes) >> 4);
-                    const int n16 = (nv + 15) / 16;
-                    for (int kk = 0; kk < n16; ++kk)
-                        mma_f16_ts(tmem + col_o(t), tmem + col_s(t) + kk * 8, vd + (uint64_t)(kk * 128), kPV,
-                                   (j > 0 || kk > 0) ? 1u : 0u);
-                    tc_commit(&sm.pv_done[t]);
-                    return true;
-                };
-                if (!mbar_wait(&sm.q_full, 0, limit)) fail = true;
-                step_tile();                                                 // nv_cur = tile 0
-                for (int t = 0; t < n_qt && !fail; ++t)
-                    if (!issue_qk(t, 0, nv_cur)) fail = true;
-                if (!fail) tc_commit(&sm.kv_empty[0]);
+                if (!mbar_wait_backoff(&sm.q_full, 0, limit)) fail = true;
+                if (!fail && !issue_qk(0)) fail = true;
+                if (!fail && n_tiles > 1 && !issue_qk(1)) fail = true;
                 for (int j = 0; j < n_tiles && !fail; ++j) {
-                    const int nv_pv = nv_cur;
-                    if (j + 1 < n_tiles) step_tile();                        // nv_cur = tile j + 1
-                    for (int t = 0; t < n_qt; ++t) {
-                        if (!issue_pv(t, j, nv_pv)) { fail = true; break; }
-                        // S_t is rewritten right behind PV_t(j), which reads P_t out of
-                        // it: MMAs from one thread execute in issue order
-                        if (j + 1 < n_tiles && !issue_qk(t, j + 1, nv_cur)) { fail = true; break; }
-                    }
-                    if (fail) break;
-                    tc_commit(&sm.v16_free[j % kNV16]);
-                    if (j + 1 < n_tiles) tc_commit(&sm.kv_empty[(j + 1) % kStages]);
+                    const int b = j & 1, vb = j % kNV16;
+                    // O_t += P_t,b V_j once the softmax wrote P and V_j is widened
+                    if (!mbar_wait_backoff(&sm.p_ready[t][b], (j >> 1) & 1, limit)) { fail = true; break; }
+                    if (!mbar_wait_backoff(&sm.v16_ready[vb], (j / kNV16) & 1, limit)) { fail = true; break; }
+                    tc_fence_after();
+                    const uint64_t vd = v_desc0 + (uint64_t)((vb * kV16Bytes) >> 4);
+#pragma unroll
+                    for (int kk = 0; kk < kBN / 16; ++kk)
+                        mma_f16_ts(tmem + col_o(t), tmem + col_s(t, b) + kk * 8, vd + (uint64_t)(kk * 128), kPV,
+                                   (j > 0 || kk > 0) ? 1u : 0u);
+                    tc_commit(&sm.pv_done[t][b]);
+                    tc_commit(&sm.kv_empty[j % kStages]);
+                    tc_commit(&sm.tile_done[vb]);
+                    // QK(j+2) reuses S_t,b right behind PV(j), which reads P out of
+                    // it: tcgen05 MMAs issued by one thread execute in issue order,
+                    // so no completion wait is needed between them.
+                    if (j + 2 < n_tiles && !issue_qk(j + 2)) { fail = true; break; }
                 }
                 // drain: all MMAs issued by this thread complete before TMEM is freed
-                tc_commit(&sm.drain);
-                if (!mbar_wait(&sm.drain, 0, limit)) fail = true;
+                tc_commit(&sm.drain[t]);
+                if (!mbar_wait_backoff(&sm.drain[t], 0, limit)) fail = true;
             }
-        } else {
-            // ---------------------------------- V widening (FP8 -> f16), 2 warps --
-            // Warp 2 widens keys [0, 64) of each tile, warp 3 keys [64, 128).  A
-            // warp step covers 8 consecutive key rows x 4 chunk columns of one
-            // 64-element block: in every 8-lane shared-memory phase the 8 rows
-            // hit 8 different 16-byte bank groups, for the swizzled reads and
-            // for both swizzled writes.
+        } else if (warp == 2) {
+            // ------------------------------------------- V widening (FP8->f16) --
+            // A warp step covers 8 consecutive key rows x 4 chunk columns of one
+            // 64-element block: in every 8-lane shared-memory phase the 8 rows hit
+            // 8 different 16-byte bank groups, for the swizzled reads and for both
+            // swizzled writes.
             constexpr int kNB = D / 64;                 // 64-element blocks per key row
-            const int r0 = (warp - 2) * 64;
             const int rl = lane & 7, cq = lane >> 3;
             for (int j = 0; j < n_tiles; ++j) {
                 const int st = j % kStages, b = j % kNV16;
                 if (!warp_wait_sleep(&sm.k_full[st], (j / kStages) & 1, limit)) { fail = true; break; }
                 if (j >= kNV16 &&
-                    !warp_wait_sleep(&sm.v16_free[b], ((j / kNV16) - 1) & 1, limit)) { fail = true; break; }
-                const int nv = tile_at(p, j0 + j).nv;
-                const int rows = min(64, ((nv + 15) & ~15) - r0);   // rows the PV MMA reads
+                    !warp_wait_sleep(&sm.tile_done[b], ((j / kNV16) - 1) & 1, limit)) { fail = true; break; }
                 const uint8_t* src = sm.v8[st];
                 uint8_t* dst = sm.v16[b];
-#pragma unroll 4
-                for (int combo = 0; combo < (64 / 8) * kNB; ++combo) {
-                    const int r = r0 + (combo / kNB) * 8 + rl;
-                    if ((combo / kNB) * 8 >= rows) break;
+    #pragma unroll 4
+                for (int combo = 0; combo < (kBN / 8) * kNB; ++combo) {
+                    const int r = (combo / kNB) * 8 + rl;
                     const int nb = combo % kNB;
                     const int c = nb * 4 + cq;                              // 16-byte chunk of the FP8 row
                     const int sc = D == 128 ? (c ^ (r & 7)) : (c ^ ((r >> 1) & 3));
@@ -533,11 +450,7 @@ attend_kernel(const __grid_constant__ AttendParams p, const __grid_constant__ CU
                         make_uint4(o[4], o[5], o[6], o[7]);
                 }
                 fence_async_smem();   // generic-proxy writes -> visible to the MMA's async proxy
-                __syncwarp();
-                if (lane == 0) {
-                    mbar_arrive(&sm.v16_ready[b]);
-                    mbar_arrive(&sm.kv_empty[st]);
-                }
+                mbar_arrive(&sm.v16_ready[b]);
             }
         }
     } else {
@@ -548,7 +461,6 @@ attend_kernel(const __grid_constant__ AttendParams p, const __grid_constant__ CU
             const int row = (warp & 3) * 32 + lane;     // TMEM lane == query row in tile
             const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
             const uint32_t t_o = tmem + lane_off + col_o(t);
-            const uint32_t t_s = tmem + lane_off + col_s(t);
             const int qrow = q0 + t * kBM + row;
             const bool row_ok = qrow < p.M;
             const float sq = row_ok ? p.q_scales[(size_t)h * p.q_scale_pitch + qrow] : 0.f;
@@ -574,18 +486,20 @@ attend_kernel(const __grid_constant__ AttendParams p, const __grid_constant__ CU
             const uint64_t c2c2 = pack2(c2, c2);
             const int log2_sv_i = ve - 127;
             for (int j = 0; j < n_tiles && !fail; ++j) {
-                const int st = j % kStages;
-                const int nv = tile_at(p, j0 + j).nv;
+                const int st = j % kStages, b = j & 1;
+                const int fi = (j0 + j) / p.tiles_per_frame;
+                const int nv = min(kBN, p.T - (j0 + j - fi * p.tiles_per_frame) * kBN);
+                const uint32_t t_s = tmem + lane_off + col_s(t, b);
                 if (!warp_wait(&sm.k_full[st], (j / kStages) & 1, limit)) { fail = true; break; }
-                if (!warp_wait(&sm.s_full[t], j & 1, limit)) { fail = true; break; }
+                if (!warp_wait(&sm.s_full[t][b], (j >> 1) & 1, limit)) { fail = true; break; }
                 tc_fence_after();
                 uint32_t sr[kBN];
 #pragma unroll
-                for (int c = 0; c < kBN / 32; ++c)
-                    if (32 * c < nv) tmem_ld32(t_s + c * 32, sr + c * 32);
+                for (int c = 0; c < kBN / 32; ++c) tmem_ld32(t_s + c * 32, sr + c * 32);
                 tc_wait_ld();
                 if (j == 0)   // the first tile sets the reference
-                    m = tile_row_max(sr, sm.sk[st], nv);
+                    m = nv == kBN ? tile_row_max<false>(sr, sm.sk[st], nv)
+                                  : tile_row_max<true>(sr, sm.sk[st], nv);
                 // single pass against the reference: p/Sv = 2^(u*c2 - m*c2 - log2 Sv).
                 // The row sum bounds every p of the tile; if some row's sum
                 // (times Sv) reaches 2^15, a p may be past f16 P range and the
@@ -596,10 +510,13 @@ attend_kernel(const __grid_constant__ AttendParams p, const __grid_constant__ CU
 #pragma unroll 1
                 for (int attempt = 0; attempt < 2; ++attempt) {
                     const float neg = -(m * c2 + log2_sv);
-                    ls = tile_exp(sr, t_s, sm.sk[st], sm.sv[st], c2c2, pack2(neg, neg), nv);
+                    ls = nv == kBN
+                             ? tile_exp<false>(sr, t_s, sm.sk[st], sm.sv[st], c2c2, pack2(neg, neg), nv)
+                             : tile_exp<true>(sr, t_s, sm.sk[st], sm.sv[st], c2c2, pack2(neg, neg), nv);
                     ls_e = (int)((__float_as_uint(ls) >> 23) & 0xff) - 127 + log2_sv_i;
                     if (attempt == 1 || !__any_sync(0xffffffffu, ls_e >= kRedoLog2)) break;
-                    const float mt = tile_row_max(sr, sm.sk[st], nv);
+                    const float mt = nv == kBN ? tile_row_max<false>(sr, sm.sk[st], nv)
+                                               : tile_row_max<true>(sr, sm.sk[st], nv);
                     const float m_new = fmaxf(m, mt);
                     const float alpha = ex2((m - m_new) * c2);
                     l *= alpha;
@@ -612,7 +529,7 @@ attend_kernel(const __grid_constant__ AttendParams p, const __grid_constant__ CU
                 // has completed and before PV(j) is issued (warp-uniform: the
                 // wait and the TMEM load/store are warp-collective).
                 if (__any_sync(0xffffffffu, o_scale != 1.f)) {
-                    if (j > 0 && !warp_wait(&sm.pv_done[t], (j - 1) & 1, limit)) { fail = true; break; }
+                    if (j > 0 && !warp_wait(&sm.pv_done[t][(j - 1) & 1], ((j - 1) >> 1) & 1, limit)) { fail = true; break; }
                     tc_fence_after();
 #pragma unroll 1
                     for (int c = 0; c < D / 32; ++c) {
@@ -627,11 +544,7 @@ attend_kernel(const __grid_constant__ AttendParams p, const __grid_constant__ CU
                 }
                 tc_wait_st();
                 tc_fence_before();
-                __syncwarp();
-                if (lane == 0) {
-                    mbar_arrive(&sm.p_ready[t]);
-                    mbar_arrive(&sm.kv_empty[st]);   // this warp's reads of the stage's scales are done
-                }
+                mbar_arrive(&sm.p_ready[t][b]);
                 // lazy move of the reference: only when this tile's row sum grew
                 // to 2^8 of it; by an exact power of two, l now, O before the next
                 // PV (after PV(j)).
@@ -642,7 +555,8 @@ attend_kernel(const __grid_constant__ AttendParams p, const __grid_constant__ CU
                     m += (float)ls_e / c2;
                 }
             }
-            if (!fail && !warp_wait(&sm.pv_done[t], (n_tiles - 1) & 1, limit)) fail = true;
+            if (!fail && !warp_wait(&sm.pv_done[t][(n_tiles - 1) & 1], ((n_tiles - 1) >> 1) & 1, limit))
+                fail = true;
             if (!fail) {
                 tc_fence_after();
                 // one split: the normalised output.  Several: this range's O

@@ -18,7 +18,7 @@ constexpr int kMaxRopeHalf = 32;   // rope_t / 2 <= 32 (frame-axis table travels
 // Attention tiling shared by the kernel and the host-side TMA descriptors:
 // 128 query rows per query tile, 64 keys per KV tile.
 constexpr int kAttendRows = 128;
-constexpr int kAttendKeys = 128;
+constexpr int kAttendKeys = 64;
 constexpr int kMaxSplit = 4;       // key-range splits of one attention call
 constexpr int kMaxDevices = 64;    // per-device one-time set-up tables
 

@@ -133,15 +133,15 @@ def test_injected_allocation_failure_returns_oom():
 
 def test_split_plan_choices_and_invariants(rtv):
     """The key-range split rtv_attend uses (host arithmetic, no device)."""
-    # full-shape layer, ring full: 12 row blocks x 40 heads, 9 frames x 24 tiles of 128 keys,
-    # 148 SMs: 480 CTAs = 3.24 waves unsplit; 4 splits of 54 tiles -> 13 waves of quarter CTAs
-    assert rtv.split_plan(480, 9 * 24, 148) == (4, 54)
-    # the same layer's first step (one frame of keys): 24 tiles allow 3 splits of 8
-    assert rtv.split_plan(480, 24, 148) == (3, 8)
-    # two frames per chunk, W=16 + pinned: 24 x 40 units, 19 x 24 tiles -> 2 splits
-    assert rtv.split_plan(960, 19 * 24, 148) == (2, 228)
-    # 704-token frames, 8 heads, 7 frames of 6 tiles: 24 units fill a fraction of the GPU
-    assert rtv.split_plan(24, 42, 148) == (4, 11)
+    # full-shape layer, ring full: 12 row blocks x 40 heads, 9 frames x 47 tiles, 148 SMs:
+    # 480 CTAs = 3.24 waves unsplit; 4 splits of <= 106 tiles -> 13 waves of quarter CTAs
+    assert rtv.split_plan(480, 9 * 47, 148) == (4, 106)
+    # the same layer's first step (one frame of keys): still 4 splits, of 12 tiles (last 11)
+    assert rtv.split_plan(480, 47, 148) == (4, 12)
+    # two frames per chunk, W=16 + pinned: 24 x 40 units, 19 x 47 tiles -> 2 splits
+    assert rtv.split_plan(960, 19 * 47, 148) == (2, 447)
+    # 704-token frames, 8 heads, 7 frames of 11 tiles: 24 units fill a fraction of the GPU
+    assert rtv.split_plan(24, 77, 148) == (4, 20)
     # too few tiles to split (fewer than 8 per split)
     assert rtv.split_plan(2, 5, 148) == (1, 5)
     assert rtv.split_plan(480, 15, 148) == (1, 15)
