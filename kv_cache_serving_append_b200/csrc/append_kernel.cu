@@ -161,7 +161,8 @@ __device__ __forceinline__ void append_rows(const AppendParams& p, int tensor,
 
         // this lane's cos/sin for the row, staged in the half-warp's slice of
         // shared memory (read back per head; 16-byte accesses, no conflicts)
-        float* cs = s_cs + ((threadIdx.x >> 4) * 2 * D) + lane16 * E;   // cos at cs, sin at cs + D
+        // [cos | sin] x [e / 4][lane][4]: the 16 lanes' float4 accesses are consecutive
+        float* cs = s_cs + ((threadIdx.x >> 4) * 2 * D) + lane16 * 4;   // cos at cs, sin at cs + D
         if (rope) {
             float cc[E], ss[E];
             if (seg == 0) {
@@ -183,8 +184,8 @@ __device__ __forceinline__ void append_rows(const AppendParams& p, int tensor,
             __syncwarp();   // the previous row's reads of this slice are done
 #pragma unroll
             for (int e = 0; e < E; e += 4) {
-                *reinterpret_cast<float4*>(cs + e) = make_float4(cc[e], cc[e + 1], cc[e + 2], cc[e + 3]);
-                *reinterpret_cast<float4*>(cs + D + e) = make_float4(ss[e], ss[e + 1], ss[e + 2], ss[e + 3]);
+                *reinterpret_cast<float4*>(cs + (e >> 2) * 64) = make_float4(cc[e], cc[e + 1], cc[e + 2], cc[e + 3]);
+                *reinterpret_cast<float4*>(cs + D + (e >> 2) * 64) = make_float4(ss[e], ss[e + 1], ss[e + 2], ss[e + 3]);
             }
             __syncwarp();
         }
@@ -226,8 +227,8 @@ __device__ __forceinline__ void append_rows(const AppendParams& p, int tensor,
                     unpack_bf16(praw, xp);
 #pragma unroll
                     for (int e = 0; e < E; e += 4) {
-                        const float4 c4 = *reinterpret_cast<const float4*>(cs + e);
-                        const float4 s4 = *reinterpret_cast<const float4*>(cs + D + e);
+                        const float4 c4 = *reinterpret_cast<const float4*>(cs + (e >> 2) * 64);
+                        const float4 s4 = *reinterpret_cast<const float4*>(cs + D + (e >> 2) * 64);
                         cc[e] = c4.x; cc[e + 1] = c4.y; cc[e + 2] = c4.z; cc[e + 3] = c4.w;
                         ss[e] = s4.x; ss[e + 1] = s4.y; ss[e + 2] = s4.z; ss[e + 3] = s4.w;
                     }
