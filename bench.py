@@ -319,6 +319,28 @@ def run_seq48(args):
     return 0
 
 
+def run_project(args):
+    """--workload project: the fused QKV projection + append on its own JSON
+    line (one GPU), beside the unfused library path it replaces."""
+    import torch
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    r = time_project(dev, args.steps, args.warmup)
+    hbm_gbs, bf16_tf, bf16_tf_sus, peak_src = load_peaks()
+    line = {"metric": "us per fused QKV projection + append (2992 x 15360 x 5120 FP8 GEMM)",
+            "value": r["fused_us"], "unit": "us/call", "n_gpus": 1, "steps": args.steps,
+            "warmup": args.warmup, "higher_is_better": False, "data": "synthetic",
+            "config": {"workload": r["workload"]},
+            "roofline": {"bound": "tensor", "achieved": r["fused_tflops"], "peak": 2.0 * bf16_tf,
+                         "unit": "TFLOP/s", "frac": r["fused_tflops"] / (2.0 * bf16_tf),
+                         "peak_source": f"{peak_src} bf16 burst x 2 (nominal fp8:bf16 ratio)",
+                         "traffic": ncu_traffic("project_kernel.cu", "project_full_shape_ncu.md"),
+                         "algorithmic_flop_per_launch": r["gemm_flop"]},
+            "unfused_us": r.get("unfused_us"), "unfused_path": r.get("unfused_path")}
+    print(json.dumps(line))
+    return 0
+
+
 def run_reference(args):
     """--impl reference: the CPU oracle as it stands, on the host cores, one
     whole full-shape layer-step per step (rank 0 only)."""
@@ -628,12 +650,14 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extra", action="store_true",
                     help="skip the long-window, multi-pass and 48-layer workloads")
-    ap.add_argument("--workload", default="layer", choices=["layer", "seq48"])
+    ap.add_argument("--workload", default="layer", choices=["layer", "seq48", "project"])
     args = ap.parse_args()
     if args.impl == "reference":
         return run_reference(args)
     if args.workload == "seq48":
         return run_seq48(args)
+    if args.workload == "project":
+        return run_project(args)
 
     import torch
     import torch.distributed as dist
