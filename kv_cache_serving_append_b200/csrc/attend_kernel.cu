@@ -14,26 +14,32 @@
 //   warp 0     TMA producer: both Q tiles once; per KV tile the K and V code
 //              tiles at (ring slot * H + head, token tile) and their scales.
 //   warps 1,3  MMA issuers, one per query tile t (warp 1 also owns TMEM).
-//              S_t,b = Q_t K_j^T (kind::f8f6f4, E4M3 x E4M3 -> f32 in TMEM,
-//              b = j mod 2: two S buffers per query tile), O_t += P_t,b V16_j
-//              (kind::f16, P read from TMEM where it overwrote S_t,b, V16
-//              from shared memory).  With two S buffers the softmax of KV tile
-//              j+1 runs while PV(j) and QK(j+2) execute.
+//              S_t = Q_t K_j^T (kind::f8f6f4, E4M3 x E4M3 -> f32 in TMEM),
+//              O_t += P_t,b V16_j (kind::f16, b = j mod 2, P read from TMEM,
+//              V16 from shared memory).  S_t(j+2) is issued as soon as the
+//              softmax has read S_t(j+1) into registers -- ahead of PV(j),
+//              which is off the softmax's critical path -- so the next scores
+//              are computed while the softmax works on the current ones.
 //   warp 2     widens the V code tile to f16 (exact) in the MN-major layout
 //              the PV MMA reads.
 //   warps 4-7  softmax of query tile 0, warps 8-11 of query tile 1; one query
 //              row per thread, the tile's 64 scores in registers, one pass
 //              per KV tile against a reference m: s*scale_k, exp2, row sum,
-//              P = p*scale_v/Sv in f16 written back over S.  The row sum
+//              P = p*scale_v/Sv in f16, kept in registers until the pass
+//              stands and then stored to P_t,b in one TMEM store.  The row sum
 //              bounds every p of the tile, so it alone decides (no per-key
 //              max): a tile is redone against its exact max only when a row
 //              sum reaches 2^15 (f16 P range), and m moves up by a power of
 //              two, with O rescaled lazily, only when a row sum reaches 2^8.
 //              The two warpgroups run concurrently.
-// TMEM columns: S_t,b at 64*(2t+b) (64 columns each), O_0 [256,256+D),
-// O_1 [384,384+D).  QK(j+2) overwrites S_t,b right after PV(j), which reads
-// P_t,b out of it, is issued: tcgen05 MMAs from one issuing thread execute in
-// order, so the write cannot overtake the read.
+// TMEM columns of query tile t: S_t [256t, 256t+64), P_t,0 and P_t,1 (f16
+// pairs, 32 columns each) [256t+64, 256t+128), O_t [256t+128, 256t+128+D).
+// S is single-buffered: QK(j+1) waits (s_free) until every softmax thread
+// has read S(j).  P is double-buffered: softmax(j) writes P_t,b only after
+// PV(j-2), its previous reader, has completed (pv_done).
+// Per-tile waits avoid integer division (frame and tile-in-frame are walked),
+// and at the end each warp's 32 output rows leave through shared memory so
+// that the global stores write whole row segments.
 //
 // Logical-to-physical frame order is resolved in the TMA coordinates: the
 // kernel receives the key set as a list of ring slots -- no gather, no copy.
@@ -74,8 +80,9 @@ constexpr uint32_t kTmemCols = 512;
 constexpr int kLazyRescaleLog2 = 8;     // move the reference when a tile's row sum reaches 2^8 of it
 constexpr int kRedoLog2 = 15;           // redo a tile whose row sum reaches 2^15 (f16 P range)
 
-__host__ __device__ constexpr uint32_t col_s(int t, int b) { return 64u * (2 * t + b); }
-__host__ __device__ constexpr uint32_t col_o(int t) { return 256u + 128u * t; }
+__host__ __device__ constexpr uint32_t col_s(int t) { return 256u * t; }
+__host__ __device__ constexpr uint32_t col_p(int t, int b) { return 256u * t + 64u + 32u * b; }
+__host__ __device__ constexpr uint32_t col_o(int t) { return 256u * t + 128u; }
 
 template <int D>
 struct Smem {
@@ -91,7 +98,7 @@ struct Smem {
     uint64_t q_full;
     uint64_t k_full[kStages];
     uint64_t kv_empty[kStages];
-    uint64_t s_full[kQT][2], p_ready[kQT][2], pv_done[kQT][2];
+    uint64_t s_full[kQT], s_free[kQT], p_ready[kQT][2], pv_done[kQT][2];
     uint64_t v16_ready[kNV16], tile_done[kNV16];
     uint64_t drain[kQT];
     uint32_t tmem_base;
@@ -200,51 +207,72 @@ __device__ __forceinline__ float tile_row_max(const uint32_t* sr, const float* s
 
 // One pass over a KV tile (the kBN scores of this thread's row in registers):
 // u = s * scale_k, x = u*c2 + neg (= (u - m)*c2 - log2 Sv for the reference
-// m), p/Sv = 2^x, P = (p/Sv) * scale_v packed to f16 pairs and written over S
-// in TMEM (keys [32c, 32c+32) -> P columns [16c, 16c+16); S is already in
-// registers).  Returns the row sum of p/Sv, which also bounds every p/Sv of
-// the tile: the caller reads from it whether the tile outgrew m.
+// m), p/Sv = 2^x, P = (p/Sv) * scale_v packed to f16 pairs in pk (key 2i and
+// 2i+1 in pk[i]).  Nothing is stored: the caller writes P once it knows the
+// pass stands and the P buffer is free, and the compiler is free to interleave
+// the whole tile's exponentials.  Returns the row sum of p/Sv, which also
+// bounds every p/Sv of the tile: the caller reads from it whether the tile
+// outgrew m.
 template <bool kMask>
-__device__ __forceinline__ float tile_exp(const uint32_t* sr, uint32_t t_s, const float* sk,
-                                          const float* sv, uint64_t c2c2, uint64_t neg2, int nv)
+__device__ __forceinline__ float tile_p(const uint32_t* sr, uint32_t* pk, const float* sk, const float* sv,
+                                        uint64_t c2c2, uint64_t neg2, int nv)
 {
     const float4* sk4 = reinterpret_cast<const float4*>(sk);
     const float4* sv4 = reinterpret_cast<const float4*>(sv);
     // independent partial row sums: short dependency chains
     uint64_t ls2[4] = {pack2(0.f, 0.f), pack2(0.f, 0.f), pack2(0.f, 0.f), pack2(0.f, 0.f)};
 #pragma unroll
-    for (int c = 0; c < kBN / 32; ++c) {
-        uint32_t pk[16];
+    for (int k4 = 0; k4 < kBN / 4; ++k4) {
+        const float4 kk = sk4[k4];
+        const float4 vv = sv4[k4];
 #pragma unroll
-        for (int k4 = 0; k4 < 8; ++k4) {
-            const float4 kk = sk4[c * 8 + k4];
-            const float4 vv = sv4[c * 8 + k4];
-#pragma unroll
-            for (int hh = 0; hh < 2; ++hh) {
-                const int k = c * 32 + 4 * k4 + 2 * hh;
-                const uint64_t u = mul2(pack2(__uint_as_float(sr[k]), __uint_as_float(sr[k + 1])),
-                                        hh ? pack2(kk.z, kk.w) : pack2(kk.x, kk.y));
-                float x0, x1;
-                unpack2(fma2(u, c2c2, neg2), x0, x1);
-                if (kMask) {
-                    if (k >= nv) x0 = -INFINITY;
-                    if (k + 1 >= nv) x1 = -INFINITY;
-                }
-                const float p0 = ex2(x0), p1 = ex2(x1);   // ex2(-inf) = 0 for masked keys
-                const uint64_t pp = pack2(p0, p1);
-                ls2[(k >> 1) & 3] = add2(ls2[(k >> 1) & 3], pp);
-                float q0, q1;
-                unpack2(mul2(pp, hh ? pack2(vv.z, vv.w) : pack2(vv.x, vv.y)), q0, q1);
-                __half2 hv = __floats2half2_rn(q0, q1);
-                pk[(4 * k4 + 2 * hh) / 2] = *reinterpret_cast<uint32_t*>(&hv);
+        for (int hh = 0; hh < 2; ++hh) {
+            const int k = 4 * k4 + 2 * hh;
+            const uint64_t u = mul2(pack2(__uint_as_float(sr[k]), __uint_as_float(sr[k + 1])),
+                                    hh ? pack2(kk.z, kk.w) : pack2(kk.x, kk.y));
+            float x0, x1;
+            unpack2(fma2(u, c2c2, neg2), x0, x1);
+            if (kMask) {
+                if (k >= nv) x0 = -INFINITY;
+                if (k + 1 >= nv) x1 = -INFINITY;
             }
+            const float p0 = ex2(x0), p1 = ex2(x1);   // ex2(-inf) = 0 for masked keys
+            const uint64_t pp = pack2(p0, p1);
+            ls2[(k >> 1) & 3] = add2(ls2[(k >> 1) & 3], pp);
+            float q0, q1;
+            unpack2(mul2(pp, hh ? pack2(vv.z, vv.w) : pack2(vv.x, vv.y)), q0, q1);
+            __half2 hv = __floats2half2_rn(q0, q1);
+            pk[k / 2] = *reinterpret_cast<uint32_t*>(&hv);
         }
-        tmem_st16(t_s + c * 16, pk);
     }
     float a, b, c, d;
     unpack2(add2(ls2[0], ls2[1]), a, b);
     unpack2(add2(ls2[2], ls2[3]), c, d);
     return (a + b) + (c + d);
+}
+
+// TMEM store of 32 columns without a compiler memory clobber: it touches no
+// generic memory, and its order against the tcgen05 waits, fences and
+// mbarrier arrives (all volatile asm) is kept.
+__device__ __forceinline__ void tmem_st32_p(uint32_t taddr, const uint32_t* r)
+{
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,"
+        "%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+        "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+        "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]),
+        "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]),
+        "r"(r[29]), "r"(r[30]), "r"(r[31]));
+}
+
+// Both phases complete (two try_waits in flight together), warp-uniform.
+__device__ __forceinline__ bool warp_wait2(uint64_t* a, uint32_t pa, uint64_t* b, uint32_t pb, long long limit)
+{
+    const bool ra = mbar_try_wait(a, pa);
+    const bool rb = mbar_try_wait(b, pb);
+    if (__all_sync(0xffffffffu, ra && rb)) return true;
+    return __all_sync(0xffffffffu, mbar_wait(a, pa, limit) && mbar_wait(b, pb, limit));
 }
 
 __device__ __forceinline__ void reg_dealloc_56() { asm volatile("setmaxnreg.dec.sync.aligned.u32 56;"); }
@@ -272,6 +300,12 @@ attend_kernel(const __grid_constant__ AttendParams p, const __grid_constant__ CU
     const int n_tiles = min(p.n_frames_keys * p.tiles_per_frame - j0, p.tiles_per_split);
     const int n_qt = min(kQT, (p.M - q0 + kBM - 1) / kBM);   // query tiles with valid rows
     const long long limit = p.wait_limit;
+    // The K/V tensor maps' box must be this kernel's KV tile: a host built
+    // against another tile size would have TMA write past the stage buffers.
+    if (p.key_tile != kBN) {
+        if (threadIdx.x == 0) atomicOr(p.err, kErrBounds);
+        return;
+    }
 #ifdef RTV_DEBUG
     // every frame of the key set must name a slot of the cache: checked before
     // any barrier, TMEM or memory is touched; the whole CTA returns alike
@@ -296,8 +330,9 @@ attend_kernel(const __grid_constant__ AttendParams p, const __grid_constant__ CU
             mbar_init(&sm.kv_empty[s], n_qt);
         }
         for (int t = 0; t < kQT; ++t) {
+            mbar_init(&sm.s_full[t], 1);
+            mbar_init(&sm.s_free[t], 128);
             for (int b = 0; b < 2; ++b) {
-                mbar_init(&sm.s_full[t][b], 1);
                 mbar_init(&sm.p_ready[t][b], 128);
                 mbar_init(&sm.pv_done[t][b], 1);
             }
@@ -338,15 +373,15 @@ attend_kernel(const __grid_constant__ AttendParams p, const __grid_constant__ CU
                 mbar_arrive_expect_tx(&sm.q_full, kQT * kQBytes);
                 for (int t = 0; t < kQT; ++t) tma_load_3d(sm.q[t], &map_q, &sm.q_full, 0, q0 + t * kBM, h);
                 int issued = 0;
-                for (int j = 0; j < n_tiles; ++j) {
+                int fi = j0 / p.tiles_per_frame, tif = j0 - fi * p.tiles_per_frame;
+                for (int j = 0; j < n_tiles; ++j, tif = (tif + 1 == p.tiles_per_frame) ? (++fi, 0) : tif + 1) {
                     const int st = j % kStages;
                     if (j >= kStages &&
                         !mbar_wait_sleep(&sm.kv_empty[st], ((j / kStages) - 1) & 1, limit)) {
                         fail = true;
                         break;
                     }
-                    const int fi = (j0 + j) / p.tiles_per_frame;
-                    const int t0 = (j0 + j - fi * p.tiles_per_frame) * kBN;
+                    const int t0 = tif * kBN;
                     const int row = key_slot(p, fi) * H + h;
                     mbar_arrive_expect_tx(&sm.k_full[st], 2 * kKVBytes + 2 * kBN * 4);
                     tma_load_3d(sm.k[st], &map_k, &sm.k_full[st], 0, t0, row);
@@ -377,39 +412,42 @@ attend_kernel(const __grid_constant__ AttendParams p, const __grid_constant__ CU
                 const uint64_t q_desc = smem_desc(smem_u32(sm.q[t]), 16, kSbo, kSw);
                 const uint64_t k_desc0 = smem_desc(smem_u32(sm.k[0]), 16, kSbo, kSw);
                 const uint64_t v_desc0 = smem_desc(smem_u32(sm.v16[0]), kBN * 128, 1024, kSwizzle128);
-                // S_t,b = Q_t K_j^T, b = j & 1, once K_j has landed
+                // S_t = Q_t K_j^T once K_j has landed
                 auto issue_qk = [&](int j) -> bool {
                     if (!mbar_wait_backoff(&sm.k_full[j % kStages], (j / kStages) & 1, limit)) return false;
                     tc_fence_after();
                     const uint64_t kd = k_desc0 + (uint64_t)(((j % kStages) * kKVBytes) >> 4);
 #pragma unroll
                     for (int kk = 0; kk < D / 32; ++kk)
-                        mma_f8_ss(tmem + col_s(t, j & 1), q_desc + (uint64_t)(kk * 2), kd + (uint64_t)(kk * 2),
+                        mma_f8_ss(tmem + col_s(t), q_desc + (uint64_t)(kk * 2), kd + (uint64_t)(kk * 2),
                                   kQK, kk > 0);
-                    tc_commit(&sm.s_full[t][j & 1]);
+                    tc_commit(&sm.s_full[t]);
                     return true;
                 };
                 if (!mbar_wait_backoff(&sm.q_full, 0, limit)) fail = true;
                 if (!fail && !issue_qk(0)) fail = true;
-                if (!fail && n_tiles > 1 && !issue_qk(1)) fail = true;
+                // S(1) once every softmax thread has read S(0)
+                if (!fail && n_tiles > 1 && (!mbar_wait(&sm.s_free[t], 0, limit) || !issue_qk(1))) fail = true;
                 for (int j = 0; j < n_tiles && !fail; ++j) {
                     const int b = j & 1, vb = j % kNV16;
-                    // O_t += P_t,b V_j once the softmax wrote P and V_j is widened
-                    if (!mbar_wait_backoff(&sm.p_ready[t][b], (j >> 1) & 1, limit)) { fail = true; break; }
+                    if (!mbar_wait(&sm.p_ready[t][b], (j >> 1) & 1, limit)) { fail = true; break; }
+                    // S(j+2) as soon as softmax(j+1) has read S(j+1), ahead of PV(j):
+                    // the next S is on the softmax's critical path, PV(j) is not
+                    if (j + 2 < n_tiles) {
+                        if (!mbar_wait(&sm.s_free[t], (j + 1) & 1, limit)) { fail = true; break; }
+                        if (!issue_qk(j + 2)) { fail = true; break; }
+                    }
+                    // O_t += P_t,b V_j (P_b written by softmax(j), V_j widened)
                     if (!mbar_wait_backoff(&sm.v16_ready[vb], (j / kNV16) & 1, limit)) { fail = true; break; }
                     tc_fence_after();
                     const uint64_t vd = v_desc0 + (uint64_t)((vb * kV16Bytes) >> 4);
 #pragma unroll
                     for (int kk = 0; kk < kBN / 16; ++kk)
-                        mma_f16_ts(tmem + col_o(t), tmem + col_s(t, b) + kk * 8, vd + (uint64_t)(kk * 128), kPV,
+                        mma_f16_ts(tmem + col_o(t), tmem + col_p(t, b) + kk * 8, vd + (uint64_t)(kk * 128), kPV,
                                    (j > 0 || kk > 0) ? 1u : 0u);
                     tc_commit(&sm.pv_done[t][b]);
                     tc_commit(&sm.kv_empty[j % kStages]);
                     tc_commit(&sm.tile_done[vb]);
-                    // QK(j+2) reuses S_t,b right behind PV(j), which reads P out of
-                    // it: tcgen05 MMAs issued by one thread execute in issue order,
-                    // so no completion wait is needed between them.
-                    if (j + 2 < n_tiles && !issue_qk(j + 2)) { fail = true; break; }
                 }
                 // drain: all MMAs issued by this thread complete before TMEM is freed
                 tc_commit(&sm.drain[t]);
@@ -423,6 +461,15 @@ attend_kernel(const __grid_constant__ AttendParams p, const __grid_constant__ CU
             // swizzled writes.
             constexpr int kNB = D / 64;                 // 64-element blocks per key row
             const int rl = lane & 7, cq = lane >> 3;
+            // Lane (rl, cq) handles rows 8i + rl, 16-byte chunk nb*4 + cq of each: the
+            // swizzle phase of those rows depends on rl only, so every address below
+            // is a per-lane base plus a compile-time offset.
+            const int sw = D == 128 ? rl : ((rl >> 1) & 3);
+            int src_off[kNB];
+#pragma unroll
+            for (int nb = 0; nb < kNB; ++nb) src_off[nb] = rl * D + (((nb * 4 + cq) ^ sw) << 4);
+            const int dst_a = rl * 128 + (((2 * cq) ^ rl) << 4);
+            const int dst_b = rl * 128 + (((2 * cq + 1) ^ rl) << 4);
             for (int j = 0; j < n_tiles; ++j) {
                 const int st = j % kStages, b = j % kNV16;
                 if (!warp_wait_sleep(&sm.k_full[st], (j / kStages) & 1, limit)) { fail = true; break; }
@@ -430,24 +477,21 @@ attend_kernel(const __grid_constant__ AttendParams p, const __grid_constant__ CU
                     !warp_wait_sleep(&sm.tile_done[b], ((j / kNV16) - 1) & 1, limit)) { fail = true; break; }
                 const uint8_t* src = sm.v8[st];
                 uint8_t* dst = sm.v16[b];
-    #pragma unroll 4
-                for (int combo = 0; combo < (kBN / 8) * kNB; ++combo) {
-                    const int r = (combo / kNB) * 8 + rl;
-                    const int nb = combo % kNB;
-                    const int c = nb * 4 + cq;                              // 16-byte chunk of the FP8 row
-                    const int sc = D == 128 ? (c ^ (r & 7)) : (c ^ ((r >> 1) & 3));
-                    const uint4 raw = *reinterpret_cast<const uint4*>(src + r * D + sc * 16);
-                    uint32_t o[8];
-                    e4m3x4_to_f16x4(raw.x, o[0], o[1]);
-                    e4m3x4_to_f16x4(raw.y, o[2], o[3]);
-                    e4m3x4_to_f16x4(raw.z, o[4], o[5]);
-                    e4m3x4_to_f16x4(raw.w, o[6], o[7]);
-                    // elements d = 16c .. 16c+15 = block nb, bytes 32*cq .. 32*cq+31 of the row
-                    uint8_t* rowp = dst + nb * (kBN * 128) + r * 128;
-                    *reinterpret_cast<uint4*>(rowp + (((2 * cq) ^ (r & 7)) << 4)) =
-                        make_uint4(o[0], o[1], o[2], o[3]);
-                    *reinterpret_cast<uint4*>(rowp + (((2 * cq + 1) ^ (r & 7)) << 4)) =
-                        make_uint4(o[4], o[5], o[6], o[7]);
+#pragma unroll 4
+                for (int i = 0; i < kBN / 8; ++i) {
+#pragma unroll
+                    for (int nb = 0; nb < kNB; ++nb) {
+                        const uint4 raw = *reinterpret_cast<const uint4*>(src + src_off[nb] + i * 8 * D);
+                        uint32_t o[8];
+                        e4m3x4_to_f16x4(raw.x, o[0], o[1]);
+                        e4m3x4_to_f16x4(raw.y, o[2], o[3]);
+                        e4m3x4_to_f16x4(raw.z, o[4], o[5]);
+                        e4m3x4_to_f16x4(raw.w, o[6], o[7]);
+                        // elements 16c .. 16c+15 (c = nb*4 + cq) = bytes 32*cq .. 32*cq+31 of block nb's row
+                        uint8_t* rowp = dst + nb * (kBN * 128) + i * 8 * 128;
+                        *reinterpret_cast<uint4*>(rowp + dst_a) = make_uint4(o[0], o[1], o[2], o[3]);
+                        *reinterpret_cast<uint4*>(rowp + dst_b) = make_uint4(o[4], o[5], o[6], o[7]);
+                    }
                 }
                 fence_async_smem();   // generic-proxy writes -> visible to the MMA's async proxy
                 mbar_arrive(&sm.v16_ready[b]);
@@ -485,18 +529,24 @@ attend_kernel(const __grid_constant__ AttendParams p, const __grid_constant__ CU
             float o_scale = 1.f;   // factor O still owes (applied before the next PV)
             const uint64_t c2c2 = pack2(c2, c2);
             const int log2_sv_i = ve - 127;
-            for (int j = 0; j < n_tiles && !fail; ++j) {
+            const uint32_t t_s = tmem + lane_off + col_s(t);
+            int tif = j0 % p.tiles_per_frame;       // KV tile index within its frame
+            for (int j = 0; j < n_tiles && !fail; ++j, tif = (tif + 1 == p.tiles_per_frame) ? 0 : tif + 1) {
                 const int st = j % kStages, b = j & 1;
-                const int fi = (j0 + j) / p.tiles_per_frame;
-                const int nv = min(kBN, p.T - (j0 + j - fi * p.tiles_per_frame) * kBN);
-                const uint32_t t_s = tmem + lane_off + col_s(t, b);
-                if (!warp_wait(&sm.k_full[st], (j / kStages) & 1, limit)) { fail = true; break; }
-                if (!warp_wait(&sm.s_full[t][b], (j >> 1) & 1, limit)) { fail = true; break; }
+                const int nv = min(kBN, p.T - tif * kBN);
+                const uint32_t t_p = tmem + lane_off + col_p(t, b);
+                if (!warp_wait2(&sm.k_full[st], (j / kStages) & 1, &sm.s_full[t], j & 1, limit)) { fail = true; break; }
                 tc_fence_after();
                 uint32_t sr[kBN];
 #pragma unroll
                 for (int c = 0; c < kBN / 32; ++c) tmem_ld32(t_s + c * 32, sr + c * 32);
                 tc_wait_ld();
+                // S is in registers: the issuer may overwrite it with the next tile's scores
+                tc_fence_before();
+                mbar_arrive(&sm.s_free[t]);
+                // P_b was last read by PV(j-2): tested now, waited for only
+                // before the P store, so the test's latency hides behind the pass
+                const bool p_free = j < 2 || mbar_test(&sm.pv_done[t][b], ((j - 2) >> 1) & 1);
                 if (j == 0)   // the first tile sets the reference
                     m = nv == kBN ? tile_row_max<false>(sr, sm.sk[st], nv)
                                   : tile_row_max<true>(sr, sm.sk[st], nv);
@@ -507,12 +557,12 @@ attend_kernel(const __grid_constant__ AttendParams p, const __grid_constant__ CU
                 // first tiles of a row).  ls_e = floor(log2(row sum * Sv)).
                 float ls = 0.f;
                 int ls_e = 0;
+                uint32_t pk[kBN / 2];
 #pragma unroll 1
                 for (int attempt = 0; attempt < 2; ++attempt) {
                     const float neg = -(m * c2 + log2_sv);
-                    ls = nv == kBN
-                             ? tile_exp<false>(sr, t_s, sm.sk[st], sm.sv[st], c2c2, pack2(neg, neg), nv)
-                             : tile_exp<true>(sr, t_s, sm.sk[st], sm.sv[st], c2c2, pack2(neg, neg), nv);
+                    ls = nv == kBN ? tile_p<false>(sr, pk, sm.sk[st], sm.sv[st], c2c2, pack2(neg, neg), nv)
+                                   : tile_p<true>(sr, pk, sm.sk[st], sm.sv[st], c2c2, pack2(neg, neg), nv);
                     ls_e = (int)((__float_as_uint(ls) >> 23) & 0xff) - 127 + log2_sv_i;
                     if (attempt == 1 || !__any_sync(0xffffffffu, ls_e >= kRedoLog2)) break;
                     const float mt = nv == kBN ? tile_row_max<false>(sr, sm.sk[st], nv)
@@ -522,9 +572,12 @@ attend_kernel(const __grid_constant__ AttendParams p, const __grid_constant__ CU
                     l *= alpha;
                     o_scale *= alpha;
                     m = m_new;
-                    tc_wait_st();   // the first pass's P stores land before they are overwritten
                 }
                 l += ls;
+                if (!__all_sync(0xffffffffu, p_free) &&
+                    !warp_wait(&sm.pv_done[t][b], ((j - 2) >> 1) & 1, limit)) { fail = true; break; }
+                tc_fence_after();
+                tmem_st32_p(t_p, pk);
                 // O owes a factor from an earlier move of m: apply it once PV(j-1)
                 // has completed and before PV(j) is issued (warp-uniform: the
                 // wait and the TMEM load/store are warp-collective).
@@ -568,37 +621,55 @@ attend_kernel(const __grid_constant__ AttendParams p, const __grid_constant__ CU
                 if (split && row_ok)
                     *reinterpret_cast<float2*>(p.part_ml + 2 * part_row) = make_float2(m * c2, l);
                 const float norm = split ? o_scale : o_scale / l;
+                // The warp's 32 rows leave through shared memory so that every
+                // global store writes whole row segments (4 rows x 128 bytes per
+                // instruction instead of 32 scattered 16-byte pieces).  The staging
+                // buffer is this query tile's Q code tile: its last reader, QK of
+                // the last KV tile, completed before PV of that tile did.
+                constexpr int kCW = Smem<D>::kQBytes / (4 * 32 * 4);   // staged columns per pass: 32 (D128), 16 (D64)
+                constexpr int kG = kCW / 4;                              // float4 groups per staged row
+                constexpr int kRpi = 32 / kG;                            // rows per warp store instruction
+                float* stg = reinterpret_cast<float*>(sm.q[t]) + (warp & 3) * (32 * kCW);
+                const int qbase = q0 + t * kBM + (warp & 3) * 32;
+                const bool bf = p.out_bf16 && !split;
+                const int gl = lane % kG;                                // float4 group this lane stores
 #pragma unroll 1
                 for (int c = 0; c < D / 32; ++c) {
                     uint32_t o[32];
                     tmem_ld32(t_o + c * 32, o);
                     tc_wait_ld();
-                    if (row_ok) {
-                        if (p.out_bf16 && !split) {
-                            __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(p.out) +
-                                                 ((size_t)qrow * H + h) * D + c * 32;
 #pragma unroll
-                            for (int i = 0; i < 32; i += 8) {
-                                uint32_t w[4];
+                    for (int hc = 0; hc < 32 / kCW; ++hc) {
+                        // row `lane` of the pass: float4 group g at slot g ^ (lane mod kG)
 #pragma unroll
-                                for (int e = 0; e < 4; ++e) {
-                                    __nv_bfloat162 a2 = __floats2bfloat162_rn(
-                                        __uint_as_float(o[i + 2 * e]) * norm,
-                                        __uint_as_float(o[i + 2 * e + 1]) * norm);
-                                    w[e] = *reinterpret_cast<uint32_t*>(&a2);
-                                }
-                                *reinterpret_cast<uint4*>(dst + i) = make_uint4(w[0], w[1], w[2], w[3]);
-                            }
-                        } else {
-                            float* dst = (split ? p.part_o + part_row * D
-                                                : reinterpret_cast<float*>(p.out) + ((size_t)qrow * H + h) * D) +
-                                         c * 32;
-#pragma unroll
-                            for (int i = 0; i < 32; i += 4)
-                                *reinterpret_cast<float4*>(dst + i) = make_float4(
-                                    __uint_as_float(o[i]) * norm, __uint_as_float(o[i + 1]) * norm,
-                                    __uint_as_float(o[i + 2]) * norm, __uint_as_float(o[i + 3]) * norm);
+                        for (int g = 0; g < kG; ++g) {
+                            const int e = hc * kCW + 4 * g;
+                            *reinterpret_cast<float4*>(stg + lane * kCW + 4 * (g ^ (lane % kG))) =
+                                make_float4(__uint_as_float(o[e]) * norm, __uint_as_float(o[e + 1]) * norm,
+                                            __uint_as_float(o[e + 2]) * norm, __uint_as_float(o[e + 3]) * norm);
                         }
+                        __syncwarp();
+#pragma unroll
+                        for (int it = 0; it < kG; ++it) {
+                            const int r = it * kRpi + lane / kG;
+                            const float4 v = *reinterpret_cast<const float4*>(stg + r * kCW + 4 * (gl ^ (r % kG)));
+                            const int qr = qbase + r;
+                            if (qr < p.M) {
+                                const int col = c * 32 + hc * kCW + 4 * gl;
+                                if (bf) {
+                                    __nv_bfloat162 a2 = __floats2bfloat162_rn(v.x, v.y);
+                                    __nv_bfloat162 b2 = __floats2bfloat162_rn(v.z, v.w);
+                                    *reinterpret_cast<uint2*>(reinterpret_cast<__nv_bfloat16*>(p.out) +
+                                                              ((size_t)qr * H + h) * D + col) =
+                                        make_uint2(*reinterpret_cast<uint32_t*>(&a2), *reinterpret_cast<uint32_t*>(&b2));
+                                } else {
+                                    float* dst = split ? p.part_o + (((size_t)blockIdx.z * p.M + qr) * H + h) * D
+                                                       : reinterpret_cast<float*>(p.out) + ((size_t)qr * H + h) * D;
+                                    *reinterpret_cast<float4*>(dst + col) = v;
+                                }
+                            }
+                        }
+                        __syncwarp();
                     }
                 }
             }

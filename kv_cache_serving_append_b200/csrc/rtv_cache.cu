@@ -282,6 +282,7 @@ rtv_status fill_attend_params(const rtv_cache* c, int layer, void* out, int out_
     p.H = c->H; p.D = c->D; p.T = c->T; p.M = n * c->T;
     p.q_scale_pitch = L.q_scale_pitch;
     p.out_bf16 = out_dtype == RTV_OUT_BF16;
+    p.key_tile = kAttendKeys;
     p.tiles_per_frame = (c->T + kAttendKeys - 1) / kAttendKeys;
     int nk = 0;
     for (int s : c->visible_slots) p.slot[nk++] = s;

@@ -80,6 +80,7 @@ struct AttendParams {
     int q_scale_pitch;
     int out_bf16;
     int n_frames_keys;             // frames in the key set
+    int key_tile;                  // keys per KV tile the tensor maps were encoded with (kAttendKeys)
     int tiles_per_frame;           // ceil(T / kAttendKeys)
     int n_split;                   // key-range splits (grid z); 1: no partials
     int tiles_per_split;           // KV tiles per split (the last may hold fewer)
