@@ -18,7 +18,12 @@
 // they are loaded into registers once per row and reused for every head.
 // The rotate-half partner of a lane's elements sits 2 lanes away in the frame
 // segment and 3 lanes away in the grid-row and grid-column segments (for the
-// supported splits), fetched with a shuffle.  Each half-warp keeps kItems
+// supported splits), fetched with a shuffle; the rotation's sign rides on the
+// staged sine.  The arithmetic runs two elements per instruction where that
+// is exact: the RoPE products and sum as f32x2 FMAs whose -0 addend and unit
+// factor are kernel parameters (nothing the compiler could fold into a fused
+// multiply-add), the quantising products as f32x2 multiplies, and the scale
+// amax/448 as a product with the reciprocal corrected by its FMA residual.  Each half-warp keeps kItems
 // loads in flight: the load of head h + kItems is issued as soon as head h is
 // done.  Every input byte is read once and every code byte written once.
 #include <cuda_bf16.h>
@@ -74,8 +79,46 @@ __device__ __forceinline__ uint2 shfl_vec(const uint2& v, int src)
     r.y = __shfl_sync(0xffffffffu, v.y, src);
     return r;
 }
-__device__ __forceinline__ uint4 xor_vec(const uint4& v, uint32_t m) { return make_uint4(v.x ^ m, v.y ^ m, v.z ^ m, v.w ^ m); }
-__device__ __forceinline__ uint2 xor_vec(const uint2& v, uint32_t m) { return make_uint2(v.x ^ m, v.y ^ m); }
+
+__device__ __forceinline__ uint64_t pack2(float a, float b)
+{
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+    return r;
+}
+// Two IEEE round-to-nearest products in one instruction (bit-identical to
+// two __fmul_rn; the products feed only the E4M3 conversion).
+__device__ __forceinline__ float2 mul2(float a, float b, float c)
+{
+    uint64_t r;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(pack2(a, b)), "l"(pack2(c, c)));
+    float2 o;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(o.x), "=f"(o.y) : "l"(r));
+    return o;
+}
+__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c)
+{
+    uint64_t r;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+    return r;
+}
+__device__ __forceinline__ void unpack2(uint64_t r, float& a, float& b)
+{
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(r));
+}
+
+// amax / 448, correctly rounded: the product with RN(1/448) corrected once by
+// its FMA residual (Markstein's correction step).  Checked against IEEE
+// division for every positive finite float from 2^-120 up; below that (a
+// subnormal quotient) the division itself is used.
+__device__ __forceinline__ float div448(float a)
+{
+    if (!(a >= 0x1p-120f)) return __fdiv_rn(a, 448.f);
+    constexpr float z = 1.0f / 448.0f;
+    const float q0 = __fmul_rn(a, z);
+    const float r = __fmaf_rn(-q0, 448.f, a);
+    return __fmaf_rn(r, z, q0);
+}
 
 // E4M3 round-to-nearest-even with saturation to +-448 (hardware cvt).
 __device__ __forceinline__ uint16_t e4m3x2(float lo, float hi)
@@ -85,20 +128,18 @@ __device__ __forceinline__ uint16_t e4m3x2(float lo, float hi)
 
 template <int E>
 __device__ __forceinline__ void store_codes(uint8_t* dst, const float* y, float inv);
+__device__ __forceinline__ uint16_t e4m3x2(float2 v) { return e4m3x2(v.x, v.y); }
 template <>
 __device__ __forceinline__ void store_codes<8>(uint8_t* dst, const float* y, float inv)
 {
-    uint32_t w0 = e4m3x2(__fmul_rn(y[0], inv), __fmul_rn(y[1], inv)) |
-                  ((uint32_t)e4m3x2(__fmul_rn(y[2], inv), __fmul_rn(y[3], inv)) << 16);
-    uint32_t w1 = e4m3x2(__fmul_rn(y[4], inv), __fmul_rn(y[5], inv)) |
-                  ((uint32_t)e4m3x2(__fmul_rn(y[6], inv), __fmul_rn(y[7], inv)) << 16);
+    uint32_t w0 = e4m3x2(mul2(y[0], y[1], inv)) | ((uint32_t)e4m3x2(mul2(y[2], y[3], inv)) << 16);
+    uint32_t w1 = e4m3x2(mul2(y[4], y[5], inv)) | ((uint32_t)e4m3x2(mul2(y[6], y[7], inv)) << 16);
     *reinterpret_cast<uint2*>(dst) = make_uint2(w0, w1);
 }
 template <>
 __device__ __forceinline__ void store_codes<4>(uint8_t* dst, const float* y, float inv)
 {
-    uint32_t w0 = e4m3x2(__fmul_rn(y[0], inv), __fmul_rn(y[1], inv)) |
-                  ((uint32_t)e4m3x2(__fmul_rn(y[2], inv), __fmul_rn(y[3], inv)) << 16);
+    uint32_t w0 = e4m3x2(mul2(y[0], y[1], inv)) | ((uint32_t)e4m3x2(mul2(y[2], y[3], inv)) << 16);
     *reinterpret_cast<uint32_t*>(dst) = w0;
 }
 
@@ -142,11 +183,12 @@ __device__ __forceinline__ void append_rows(const AppendParams& p, int tensor,
     const bool first_half = in_seg < seg_half;
     const int j0 = first_half ? in_seg : in_seg - seg_half;
     const int partner = (lane & 16) | (first_half ? lane16 + seg_half / E : lane16 - seg_half / E);
-    // x'[j] = x[j]c - x[j+n/2]s (first half) = x[j]c + (-x[j+n/2])s: the
-    // partner's value is negated by flipping its bf16 sign bits (exact).
-    const uint32_t neg_partner = first_half ? 0x80008000u : 0u;
+    // x'[j] = x[j]c - x[j+n/2]s (first half) = x[j]c + x[j+n/2](-s): the sign
+    // goes with the staged sine (fl(x(-s)) = -fl(xs) exactly).
+    const float sin_sign = first_half ? -1.f : 1.f;
 
     const uint16_t* src = p.src[tensor];
+    const uint64_t mz2 = pack2(p.neg_zero, p.neg_zero), one2 = pack2(p.one, p.one);
     // Rows are visited grid-stride; the trip count is the same for the two
     // half-warps of a warp only if both have a row, so the loop runs while
     // either has one (full-warp shuffles need all 32 lanes) and the other
@@ -185,7 +227,8 @@ __device__ __forceinline__ void append_rows(const AppendParams& p, int tensor,
 #pragma unroll
             for (int e = 0; e < E; e += 4) {
                 *reinterpret_cast<float4*>(cs + (e >> 2) * 64) = make_float4(cc[e], cc[e + 1], cc[e + 2], cc[e + 3]);
-                *reinterpret_cast<float4*>(cs + D + (e >> 2) * 64) = make_float4(ss[e], ss[e + 1], ss[e + 2], ss[e + 3]);
+                *reinterpret_cast<float4*>(cs + D + (e >> 2) * 64) =
+                    make_float4(sin_sign * ss[e], sin_sign * ss[e + 1], sin_sign * ss[e + 2], sin_sign * ss[e + 3]);
             }
             __syncwarp();
         }
@@ -222,7 +265,7 @@ __device__ __forceinline__ void append_rows(const AppendParams& p, int tensor,
                 float y[E];
                 unpack_bf16(cur, y);
                 if (rope) {
-                    const V praw = xor_vec(shfl_vec(cur, partner), neg_partner);
+                    const V praw = shfl_vec(cur, partner);
                     float xp[E], cc[E], ss[E];
                     unpack_bf16(praw, xp);
 #pragma unroll
@@ -232,9 +275,17 @@ __device__ __forceinline__ void append_rows(const AppendParams& p, int tensor,
                         cc[e] = c4.x; cc[e + 1] = c4.y; cc[e + 2] = c4.z; cc[e + 3] = c4.w;
                         ss[e] = s4.x; ss[e + 1] = s4.y; ss[e + 2] = s4.z; ss[e + 3] = s4.w;
                     }
+                    // fl(fl(y c) + fl(xp s)), two elements per instruction: each
+                    // product is an FMA with a -0 addend and the sum an FMA with a
+                    // unit factor, both known only at run time (kernel parameters),
+                    // so no step can be folded into a fused multiply-add and every
+                    // operation rounds once, exactly as in the scalar form.
 #pragma unroll
-                    for (int e = 0; e < E; ++e)
-                        y[e] = __fadd_rn(__fmul_rn(y[e], cc[e]), __fmul_rn(xp[e], ss[e]));
+                    for (int e = 0; e < E; e += 2) {
+                        const uint64_t t1 = fma2(pack2(y[e], y[e + 1]), pack2(cc[e], cc[e + 1]), mz2);
+                        const uint64_t t2 = fma2(pack2(xp[e], xp[e + 1]), pack2(ss[e], ss[e + 1]), mz2);
+                        unpack2(fma2(t1, one2, t2), y[e], y[e + 1]);
+                    }
                 }
                 float amax = 0.f;
 #pragma unroll
@@ -246,7 +297,7 @@ __device__ __forceinline__ void append_rows(const AppendParams& p, int tensor,
                 const float inv = amax > 0.f ? __fdiv_rn(448.f, amax) : 0.f;
                 store_codes<E>(dst + (size_t)h * dst_step, y, inv);
                 if (lane16 == 0) {
-                    const float scale = __fdiv_rn(amax, 448.f);
+                    const float scale = div448(amax);
                     sdst[(size_t)h * sdst_step] = scale;
                     if (tensor == 2) atomicMax(&s_vmax[frame][h], __float_as_uint(scale));
                 }

@@ -239,6 +239,8 @@ void fill_append_params(const rtv_cache* c, int layer, const void* q, const void
 {
     const rtv_layer_layout& L = c->layout[layer];
     std::memset(&p, 0, sizeof p);
+    p.neg_zero = -0.0f;
+    p.one = 1.0f;
     p.src[0] = static_cast<const uint16_t*>(q);
     p.src[1] = static_cast<const uint16_t*>(k);
     p.src[2] = static_cast<const uint16_t*>(v);

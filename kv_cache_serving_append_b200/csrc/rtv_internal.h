@@ -65,6 +65,7 @@ struct AppendParams {
     unsigned int seq;              // append sequence number (V-scale max tag)
     int n_slots;                   // slots of the cache (debug builds check against it)
     unsigned int* err;             // device error word
+    float neg_zero, one;           // -0.0f and 1.0f, as run-time values (see the RoPE in append_kernel.cu)
     int slot[kMaxFrames];          // ring slot of each staged frame
     float t_table[kMaxFrames][2][kMaxRopeHalf];   // frame-axis cos/sin per staged frame
     const DeviceRing* ring;        // non-null: take seq, slot and t_table from here
