@@ -689,31 +689,43 @@ attend_kernel(const __grid_constant__ AttendParams p, const __grid_constant__ CU
 // Merge of the key-range splits: one warp per (query row, head).  Split s
 // holds O_s = sum_{keys in s} 2^(x - e_s) v (unnormalised) and l_s = sum 2^(x
 // - e_s) against its own reference exponent e_s; out = sum_s 2^(e_s - e) O_s
-// / sum_s 2^(e_s - e) l_s with e = max_s e_s (the online-softmax merge).
-template <int D>
+// / sum_s 2^(e_s - e) l_s with e = max_s e_s (the online-softmax merge).  The
+// split count is a template parameter, so every split's loads are in flight
+// together.
+static_assert(kMaxSplit >= 2 && kMaxSplit <= 4, "combine_kernel is instantiated for 2, 3 and 4 splits");
+template <int D, int S>
 __global__ void __launch_bounds__(256) combine_kernel(const AttendParams p)
 {
     const int warp = (blockIdx.x * 256 + threadIdx.x) >> 5;
     const int lane = threadIdx.x & 31;
     if (warp >= p.M * p.H) return;
     const size_t stride = (size_t)p.M * p.H;          // rows of one split
-    float e = -INFINITY;
-    for (int s = 0; s < p.n_split; ++s) e = fmaxf(e, p.part_ml[2 * (s * stride + warp)]);
     constexpr int kV = D / 32;                          // elements per lane
-    float acc[kV] = {};
-    float lsum = 0.f;
-    for (int s = 0; s < p.n_split; ++s) {
-        const float2 ml = *reinterpret_cast<const float2*>(p.part_ml + 2 * (s * stride + warp));
-        const float w = exp2f(ml.x - e);
-        lsum += w * ml.y;
+    float2 ml[S];
+    float v[S][kV];
+#pragma unroll
+    for (int s = 0; s < S; ++s) {
+        ml[s] = *reinterpret_cast<const float2*>(p.part_ml + 2 * (s * stride + warp));
         const float* src = p.part_o + (s * stride + warp) * D + lane * kV;
         if constexpr (kV == 4) {
-            const float4 v = *reinterpret_cast<const float4*>(src);
-            acc[0] += w * v.x; acc[1] += w * v.y; acc[2] += w * v.z; acc[3] += w * v.w;
+            const float4 x = __ldcs(reinterpret_cast<const float4*>(src));
+            v[s][0] = x.x; v[s][1] = x.y; v[s][2] = x.z; v[s][3] = x.w;
         } else {
-            const float2 v = *reinterpret_cast<const float2*>(src);
-            acc[0] += w * v.x; acc[1] += w * v.y;
+            const float2 x = __ldcs(reinterpret_cast<const float2*>(src));
+            v[s][0] = x.x; v[s][1] = x.y;
         }
+    }
+    float e = -INFINITY;
+#pragma unroll
+    for (int s = 0; s < S; ++s) e = fmaxf(e, ml[s].x);
+    float acc[kV] = {};
+    float lsum = 0.f;
+#pragma unroll
+    for (int s = 0; s < S; ++s) {
+        const float w = exp2f(ml[s].x - e);
+        lsum += w * ml[s].y;
+#pragma unroll
+        for (int i = 0; i < kV; ++i) acc[i] += w * v[s][i];
     }
     const float inv = 1.f / lsum;
     if (p.out_bf16) {
@@ -723,8 +735,10 @@ __global__ void __launch_bounds__(256) combine_kernel(const AttendParams p)
             *reinterpret_cast<__nv_bfloat162*>(dst + i) = __floats2bfloat162_rn(acc[i] * inv, acc[i + 1] * inv);
     } else {
         float* dst = reinterpret_cast<float*>(p.out) + (size_t)warp * D + lane * kV;
-#pragma unroll
-        for (int i = 0; i < kV; ++i) dst[i] = acc[i] * inv;
+        if constexpr (kV == 4)
+            __stcs(reinterpret_cast<float4*>(dst), make_float4(acc[0] * inv, acc[1] * inv, acc[2] * inv, acc[3] * inv));
+        else
+            __stcs(reinterpret_cast<float2*>(dst), make_float2(acc[0] * inv, acc[1] * inv));
     }
 }
 
@@ -759,7 +773,12 @@ cudaError_t launch(const AttendParams& p, const CUtensorMap* maps, cudaStream_t 
     attend_kernel<D><<<grid, kThreads, smem, stream>>>(p, maps[0], maps[1], maps[2], maps[3], maps[4]);
     if (p.n_split > 1) {
         const long long warps = (long long)p.M * p.H;
-        combine_kernel<D><<<(unsigned)((warps + 7) / 8), 256, 0, stream>>>(p);
+        const unsigned blocks = (unsigned)((warps + 7) / 8);
+        switch (p.n_split) {
+            case 2: combine_kernel<D, 2><<<blocks, 256, 0, stream>>>(p); break;
+            case 3: combine_kernel<D, 3><<<blocks, 256, 0, stream>>>(p); break;
+            default: combine_kernel<D, 4><<<blocks, 256, 0, stream>>>(p); break;
+        }
     }
     return cudaGetLastError();
 }
