@@ -23,7 +23,7 @@ def cuda_ok() -> bool:
 
 @pytest.fixture(scope="session")
 def gpu():
-    """Skip-free guard: a test marked gpu must run on a GPU machine; fail loudly."""
+    """Skip-free guard: a test marked gpu must run on a GPU; fail loudly."""
     import torch
     if not torch.cuda.is_available():
         pytest.fail("test marked gpu needs a CUDA device")
