@@ -10,22 +10,20 @@
 //
 // Work split: blockIdx.y picks Q, K or V; a half-warp (16 lanes) owns one
 // token row at a time (grid-stride over the chunk's rows) and walks that
-// row's heads.  A (row, head) item is 2*D bytes of bf16: lane i loads D/16
-// contiguous elements (16 bytes at D = 128), so the 16 lanes read the item in
-// full 32-byte sectors, and the H items of a row are one contiguous stretch
-// of memory.  The RoPE cos/sin a lane needs depend only on the row (its
-// frame, grid row and grid column) and on the lane's place in head_dim, so
-// they are loaded into registers once per row and reused for every head.
-// The rotate-half partner of a lane's elements sits 2 lanes away in the frame
-// segment and 3 lanes away in the grid-row and grid-column segments (for the
-// supported splits), fetched with a shuffle; the rotation's sign rides on the
-// staged sine.  The arithmetic runs two elements per instruction where that
-// is exact: the RoPE products and sum as f32x2 FMAs whose -0 addend and unit
-// factor are kernel parameters (nothing the compiler could fold into a fused
-// multiply-add), the quantising products as f32x2 multiplies, and the scale
-// amax/448 as a product with the reciprocal corrected by its FMA residual.  Each half-warp keeps kItems
-// loads in flight: the load of head h + kItems is issued as soon as head h is
-// done.  Every input byte is read once and every code byte written once.
+// row's heads, keeping kItems loads in flight (the load of head h + kItems is
+// issued as soon as head h is done).  For V, lane i loads the D/16 contiguous
+// elements [D/16*i, D/16*(i+1)) of a (row, head) item (16 bytes at D = 128),
+// so the item is read in full sectors.  For Q and K, lane i holds D/32
+// rotation pairs (j, j + n/2) of one RoPE segment, both members loaded by
+// itself: the rotation needs no shuffle, and the lane's D/32 cos/sin pairs,
+// which depend only on the row, stay in registers for all of the row's heads.
+// The arithmetic keeps the library's rounding order bit for bit while issuing
+// two elements per instruction where that is exact: the RoPE products and sum
+// as f32x2 FMAs whose -0 addend and unit factor are kernel parameters (nothing
+// the compiler could fold into a fused multiply-add), the quantising products
+// as f32x2 multiplies, and the scale amax/448 as a product with the
+// reciprocal corrected by its FMA residual.  Every input byte is read once and
+// every code byte written once.
 #include <cuda_bf16.h>
 #include <cuda_fp8.h>
 
@@ -46,6 +44,8 @@ template <>
 struct Vec<8> { using T = uint4; };
 template <>
 struct Vec<4> { using T = uint2; };
+template <>
+struct Vec<2> { using T = uint32_t; };
 
 __device__ __forceinline__ void unpack_bf16(const uint4& v, float* x)
 {
@@ -63,21 +63,10 @@ __device__ __forceinline__ void unpack_bf16(const uint2& v, float* x)
     x[2] = __uint_as_float(v.y << 16);
     x[3] = __uint_as_float(v.y & 0xffff0000u);
 }
-__device__ __forceinline__ uint4 shfl_vec(const uint4& v, int src)
+__device__ __forceinline__ void unpack_bf16(const uint32_t& v, float* x)
 {
-    uint4 r;
-    r.x = __shfl_sync(0xffffffffu, v.x, src);
-    r.y = __shfl_sync(0xffffffffu, v.y, src);
-    r.z = __shfl_sync(0xffffffffu, v.z, src);
-    r.w = __shfl_sync(0xffffffffu, v.w, src);
-    return r;
-}
-__device__ __forceinline__ uint2 shfl_vec(const uint2& v, int src)
-{
-    uint2 r;
-    r.x = __shfl_sync(0xffffffffu, v.x, src);
-    r.y = __shfl_sync(0xffffffffu, v.y, src);
-    return r;
+    x[0] = __uint_as_float(v << 16);
+    x[1] = __uint_as_float(v & 0xffff0000u);
 }
 
 __device__ __forceinline__ uint64_t pack2(float a, float b)
@@ -143,52 +132,20 @@ __device__ __forceinline__ void store_codes<4>(uint8_t* dst, const float* y, flo
     *reinterpret_cast<uint32_t*>(dst) = w0;
 }
 
-// E consecutive floats from a 16-byte aligned address.
-template <int E>
-__device__ __forceinline__ void load_vec(const float* p, float* x)
-{
-#pragma unroll
-    for (int i = 0; i < E; i += 4) {
-        const float4 v = __ldg(reinterpret_cast<const float4*>(p + i));
-        x[i] = v.x; x[i + 1] = v.y; x[i + 2] = v.z; x[i + 3] = v.w;
-    }
-}
-
-// One tensor's rows (Q and K: ROPE; V: not rotated).  D = head_dim, E = D / 16
-// elements per lane.
-template <int D, bool ROPE>
-__device__ __forceinline__ void append_rows(const AppendParams& p, int tensor,
-                                            unsigned int (*s_vmax)[kMaxHeads], float* s_cs)
+// V: lane i of a half-warp holds the E = D/16 contiguous elements
+// [E*i, E*i + E) of a (row, head) item -- 16 bytes at D = 128 -- so the 16
+// lanes read the item in full 32-byte sectors.  The largest scale of every
+// (frame, head) is kept in shared memory for the attention's Sv.
+template <int D>
+__device__ __forceinline__ void append_rows_v(const AppendParams& p, unsigned int (*s_vmax)[kMaxHeads])
 {
     constexpr int E = D / 16;
     using V = typename Vec<E>::T;
-    constexpr bool rope = ROPE;
+    constexpr int tensor = 2;
     const int H = p.H, T = p.T;
     const int n_rows = p.n_frames * T;
-    const int ht = p.n_t / 2, hh = p.n_h / 2, hw = p.n_w / 2;
-
     const int lane16 = threadIdx.x & 15;
-    const int lane = threadIdx.x & 31;
-
-    // Fixed per lane: RoPE segment of its E elements (0 = frame, 1 = grid
-    // row, 2 = grid column), pair index of the first one, which half of the
-    // pair it holds, and its partner lane.
-    int seg = 0, seg_half = ht, seg_lo = 0;
-    if (lane16 * E >= p.n_t + p.n_h) {
-        seg = 2; seg_half = hw; seg_lo = p.n_t + p.n_h;
-    } else if (lane16 * E >= p.n_t) {
-        seg = 1; seg_half = hh; seg_lo = p.n_t;
-    }
-    const int in_seg = lane16 * E - seg_lo;
-    const bool first_half = in_seg < seg_half;
-    const int j0 = first_half ? in_seg : in_seg - seg_half;
-    const int partner = (lane & 16) | (first_half ? lane16 + seg_half / E : lane16 - seg_half / E);
-    // x'[j] = x[j]c - x[j+n/2]s (first half) = x[j]c + x[j+n/2](-s): the sign
-    // goes with the staged sine (fl(x(-s)) = -fl(xs) exactly).
-    const float sin_sign = first_half ? -1.f : 1.f;
-
     const uint16_t* src = p.src[tensor];
-    const uint64_t mz2 = pack2(p.neg_zero, p.neg_zero), one2 = pack2(p.one, p.one);
     // Rows are visited grid-stride; the trip count is the same for the two
     // half-warps of a warp only if both have a row, so the loop runs while
     // either has one (full-warp shuffles need all 32 lanes) and the other
@@ -201,59 +158,16 @@ __device__ __forceinline__ void append_rows(const AppendParams& p, int tensor,
         const int frame = row_ok ? row / T : 0;
         const int tok = row_ok ? row - frame * T : 0;
 
-        // this lane's cos/sin for the row, staged in the half-warp's slice of
-        // shared memory (read back per head; 16-byte accesses, no conflicts)
-        // [cos | sin] x [e / 4][lane][4]: the 16 lanes' float4 accesses are consecutive
-        float* cs = s_cs + ((threadIdx.x >> 4) * 2 * D) + lane16 * 4;   // cos at cs, sin at cs + D
-        if (rope) {
-            float cc[E], ss[E];
-            if (seg == 0) {
-                const float (*tt)[kMaxRopeHalf] = p.ring ? p.ring->t_table[frame] : p.t_table[frame];
-#pragma unroll
-                for (int e = 0; e < E; ++e) {
-                    cc[e] = tt[0][j0 + e];
-                    ss[e] = tt[1][j0 + e];
-                }
-            } else if (seg == 1) {
-                const float* t = p.h_table + (size_t)(tok / p.grid_w) * 2 * hh;
-                load_vec<E>(t + j0, cc);
-                load_vec<E>(t + hh + j0, ss);
-            } else {
-                const float* t = p.w_table + (size_t)(tok % p.grid_w) * 2 * hw;
-                load_vec<E>(t + j0, cc);
-                load_vec<E>(t + hw + j0, ss);
-            }
-            __syncwarp();   // the previous row's reads of this slice are done
-#pragma unroll
-            for (int e = 0; e < E; e += 4) {
-                *reinterpret_cast<float4*>(cs + (e >> 2) * 64) = make_float4(cc[e], cc[e + 1], cc[e + 2], cc[e + 3]);
-                *reinterpret_cast<float4*>(cs + D + (e >> 2) * 64) =
-                    make_float4(sin_sign * ss[e], sin_sign * ss[e + 1], sin_sign * ss[e + 2], sin_sign * ss[e + 3]);
-            }
-            __syncwarp();
-        }
-
         const V* item = reinterpret_cast<const V*>(src + (size_t)row * H * D + lane16 * E);
         V raw[kItems];
 #pragma unroll
         for (int u = 0; u < kItems; ++u) raw[u] = (row_ok && u < H) ? __ldcs(item + (size_t)u * (D / E)) : V{};
 
         // destination of head 0 of this row, and the step from one head to the next
-        uint8_t* dst;
-        float* sdst;
-        size_t dst_step, sdst_step;
-        if (tensor == 0) {
-            dst = p.q_codes + (size_t)row * D + lane16 * E;
-            sdst = p.q_scales + row;
-            dst_step = (size_t)p.q_rows * D;
-            sdst_step = p.q_scale_pitch;
-        } else {
-            const int slot = p.ring ? p.ring->staged_slot[frame] : p.slot[frame];
-            dst = p.kv_codes[tensor - 1] + ((size_t)slot * H * T + tok) * D + lane16 * E;
-            sdst = p.kv_scales[tensor - 1] + (size_t)slot * H * p.scale_pitch + tok;
-            dst_step = (size_t)T * D;
-            sdst_step = p.scale_pitch;
-        }
+        const int slot = p.ring ? p.ring->staged_slot[frame] : p.slot[frame];
+        uint8_t* dst = p.kv_codes[tensor - 1] + ((size_t)slot * H * T + tok) * D + lane16 * E;
+        float* sdst = p.kv_scales[tensor - 1] + (size_t)slot * H * p.scale_pitch + tok;
+        const size_t dst_step = (size_t)T * D, sdst_step = p.scale_pitch;
 
         for (int h0 = 0; h0 < H; h0 += kItems) {
 #pragma unroll
@@ -264,29 +178,6 @@ __device__ __forceinline__ void append_rows(const AppendParams& p, int tensor,
                 if (row_ok && h + kItems < H) raw[u] = __ldcs(item + (size_t)(h + kItems) * (D / E));
                 float y[E];
                 unpack_bf16(cur, y);
-                if (rope) {
-                    const V praw = shfl_vec(cur, partner);
-                    float xp[E], cc[E], ss[E];
-                    unpack_bf16(praw, xp);
-#pragma unroll
-                    for (int e = 0; e < E; e += 4) {
-                        const float4 c4 = *reinterpret_cast<const float4*>(cs + (e >> 2) * 64);
-                        const float4 s4 = *reinterpret_cast<const float4*>(cs + D + (e >> 2) * 64);
-                        cc[e] = c4.x; cc[e + 1] = c4.y; cc[e + 2] = c4.z; cc[e + 3] = c4.w;
-                        ss[e] = s4.x; ss[e + 1] = s4.y; ss[e + 2] = s4.z; ss[e + 3] = s4.w;
-                    }
-                    // fl(fl(y c) + fl(xp s)), two elements per instruction: each
-                    // product is an FMA with a -0 addend and the sum an FMA with a
-                    // unit factor, both known only at run time (kernel parameters),
-                    // so no step can be folded into a fused multiply-add and every
-                    // operation rounds once, exactly as in the scalar form.
-#pragma unroll
-                    for (int e = 0; e < E; e += 2) {
-                        const uint64_t t1 = fma2(pack2(y[e], y[e + 1]), pack2(cc[e], cc[e + 1]), mz2);
-                        const uint64_t t2 = fma2(pack2(xp[e], xp[e + 1]), pack2(ss[e], ss[e + 1]), mz2);
-                        unpack2(fma2(t1, one2, t2), y[e], y[e + 1]);
-                    }
-                }
                 float amax = 0.f;
 #pragma unroll
                 for (int e = 0; e < E; ++e) amax = fmaxf(amax, fabsf(y[e]));
@@ -299,8 +190,130 @@ __device__ __forceinline__ void append_rows(const AppendParams& p, int tensor,
                 if (lane16 == 0) {
                     const float scale = div448(amax);
                     sdst[(size_t)h * sdst_step] = scale;
-                    if (tensor == 2) atomicMax(&s_vmax[frame][h], __float_as_uint(scale));
+                    atomicMax(&s_vmax[frame][h], __float_as_uint(scale));
                 }
+            }
+        }
+    }
+}
+
+// Q and K.  Lane i of a half-warp holds E/2 rotation pairs (j, j + n/2) of one
+// RoPE segment -- the pairs E/2*i .. E/2*i + E/2 - 1 in segment order (frame,
+// grid row, grid column) -- so both members of every pair are its own: two
+// E/2-element loads per (row, head) item, no shuffle, and one cos/sin pair per
+// rotation pair for the whole row, held in registers.
+//   x'[j]       = fl(fl(x[j] c) + fl(x[j+n/2] (-s)))   (= x[j] c - x[j+n/2] s)
+//   x'[j + n/2] = fl(fl(x[j+n/2] c) + fl(x[j] s))
+// two elements per f32x2 FMA (the -0 addend and unit factor are parameters).
+template <int D>
+__device__ __forceinline__ void append_rows_rope(const AppendParams& p, int tensor)
+{
+    constexpr int E = D / 16;
+    constexpr int P = E / 2;                 // rotation pairs per lane
+    using HV = typename Vec<P>::T;
+    const int H = p.H, T = p.T;
+    const int n_rows = p.n_frames * T;
+    const int pt = p.n_t / 2, ph = p.n_h / 2, pw = p.n_w / 2;
+    const int lane16 = threadIdx.x & 15;
+
+    const int pq = lane16 * P;               // first pair (global pair order) of this lane
+    int seg = 0, half = pt, r0 = pq, seg_lo = 0;
+    if (pq >= pt + ph) {
+        seg = 2; half = pw; r0 = pq - pt - ph; seg_lo = p.n_t + p.n_h;
+    } else if (pq >= pt) {
+        seg = 1; half = ph; r0 = pq - pt; seg_lo = p.n_t;
+    }
+    const int ea = seg_lo + r0, eb = ea + half;   // element offsets of the two runs
+    const uint64_t mz2 = pack2(p.neg_zero, p.neg_zero), one2 = pack2(p.one, p.one);
+
+    const uint16_t* src = p.src[tensor];
+    const int stride = gridDim.x * kGroups;
+    const int row_pair0 = blockIdx.x * kGroups + ((threadIdx.x >> 4) & ~1);
+    for (int rbase = row_pair0; rbase < n_rows; rbase += stride) {
+        const int row = rbase + ((threadIdx.x >> 4) & 1);
+        const bool row_ok = row < n_rows;
+        const int frame = row_ok ? row / T : 0;
+        const int tok = row_ok ? row - frame * T : 0;
+
+        float cc[P], ss[P];
+        if (seg == 0) {
+            const float (*tt)[kMaxRopeHalf] = p.ring ? p.ring->t_table[frame] : p.t_table[frame];
+#pragma unroll
+            for (int k = 0; k < P; ++k) {
+                cc[k] = tt[0][r0 + k];
+                ss[k] = tt[1][r0 + k];
+            }
+        } else {
+            const float* t = seg == 1 ? p.h_table + (size_t)(tok / p.grid_w) * 2 * ph
+                                      : p.w_table + (size_t)(tok % p.grid_w) * 2 * pw;
+#pragma unroll
+            for (int k = 0; k < P; ++k) {
+                cc[k] = __ldg(t + r0 + k);
+                ss[k] = __ldg(t + half + r0 + k);
+            }
+        }
+
+        const uint16_t* item = src + (size_t)row * H * D;
+        HV ra[kItems], rb[kItems];
+#pragma unroll
+        for (int u = 0; u < kItems; ++u) {
+            ra[u] = (row_ok && u < H) ? __ldcs(reinterpret_cast<const HV*>(item + u * D + ea)) : HV{};
+            rb[u] = (row_ok && u < H) ? __ldcs(reinterpret_cast<const HV*>(item + u * D + eb)) : HV{};
+        }
+
+        uint8_t* dst;
+        float* sdst;
+        size_t dst_step, sdst_step;
+        if (tensor == 0) {
+            dst = p.q_codes + (size_t)row * D;
+            sdst = p.q_scales + row;
+            dst_step = (size_t)p.q_rows * D;
+            sdst_step = p.q_scale_pitch;
+        } else {
+            const int slot = p.ring ? p.ring->staged_slot[frame] : p.slot[frame];
+            dst = p.kv_codes[tensor - 1] + ((size_t)slot * H * T + tok) * D;
+            sdst = p.kv_scales[tensor - 1] + (size_t)slot * H * p.scale_pitch + tok;
+            dst_step = (size_t)T * D;
+            sdst_step = p.scale_pitch;
+        }
+
+        for (int h0 = 0; h0 < H; h0 += kItems) {
+#pragma unroll
+            for (int u = 0; u < kItems; ++u) {
+                const int h = h0 + u;
+                const HV ca = ra[u], cb = rb[u];
+                if (row_ok && h + kItems < H) {
+                    ra[u] = __ldcs(reinterpret_cast<const HV*>(item + (h + kItems) * D + ea));
+                    rb[u] = __ldcs(reinterpret_cast<const HV*>(item + (h + kItems) * D + eb));
+                }
+                float xa[P], xb[P], ya[P], yb[P];
+                unpack_bf16(ca, xa);
+                unpack_bf16(cb, xb);
+#pragma unroll
+                for (int k = 0; k < P; ++k) {
+                    const uint64_t t1 = fma2(pack2(xa[k], xb[k]), pack2(cc[k], cc[k]), mz2);
+                    const uint64_t t2 = fma2(pack2(xb[k], xa[k]), pack2(-ss[k], ss[k]), mz2);
+                    unpack2(fma2(t1, one2, t2), ya[k], yb[k]);
+                }
+                float amax = 0.f;
+#pragma unroll
+                for (int k = 0; k < P; ++k) amax = fmaxf(amax, fmaxf(fabsf(ya[k]), fabsf(yb[k])));
+#pragma unroll
+                for (int o = 8; o >= 1; o >>= 1)
+                    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+                if (!row_ok || h >= H) continue;
+                const float inv = amax > 0.f ? __fdiv_rn(448.f, amax) : 0.f;
+                uint8_t* d = dst + (size_t)h * dst_step;
+                if constexpr (P == 4) {
+                    *reinterpret_cast<uint32_t*>(d + ea) =
+                        e4m3x2(mul2(ya[0], ya[1], inv)) | ((uint32_t)e4m3x2(mul2(ya[2], ya[3], inv)) << 16);
+                    *reinterpret_cast<uint32_t*>(d + eb) =
+                        e4m3x2(mul2(yb[0], yb[1], inv)) | ((uint32_t)e4m3x2(mul2(yb[2], yb[3], inv)) << 16);
+                } else {
+                    *reinterpret_cast<uint16_t*>(d + ea) = e4m3x2(mul2(ya[0], ya[1], inv));
+                    *reinterpret_cast<uint16_t*>(d + eb) = e4m3x2(mul2(yb[0], yb[1], inv));
+                }
+                if (lane16 == 0) sdst[(size_t)h * sdst_step] = div448(amax);
             }
         }
     }
@@ -310,7 +323,6 @@ template <int D>
 __global__ void __launch_bounds__(kThreads, 4) append_kernel(const __grid_constant__ AppendParams p)
 {
     __shared__ unsigned int s_vmax[kMaxFrames][kMaxHeads];   // V only: largest scale per (frame, head)
-    __shared__ __align__(16) float s_cs[kGroups * 2 * D];      // Q, K: per half-warp cos | sin of its row
     const int tensor = blockIdx.y;             // 0 = Q, 1 = K, 2 = V
     const int H = p.H;
 #ifdef RTV_DEBUG
@@ -330,7 +342,7 @@ __global__ void __launch_bounds__(kThreads, 4) append_kernel(const __grid_consta
     if (tensor == 2) {
         for (int i = threadIdx.x; i < p.n_frames * H; i += kThreads) s_vmax[i / H][i % H] = 0u;
         __syncthreads();
-        append_rows<D, false>(p, tensor, s_vmax, s_cs);
+        append_rows_v<D>(p, s_vmax);
         __syncthreads();
         const unsigned int seq = p.ring ? p.ring->seq : p.seq;
         for (int i = threadIdx.x; i < p.n_frames * H; i += kThreads) {
@@ -340,7 +352,7 @@ __global__ void __launch_bounds__(kThreads, 4) append_kernel(const __grid_consta
             atomicMax(&p.v_scale_max[(size_t)slot * H + h], tag);
         }
     } else {
-        append_rows<D, true>(p, tensor, s_vmax, s_cs);
+        append_rows_rope<D>(p, tensor);
     }
 }
 
