@@ -141,7 +141,8 @@ def test_several_denoising_passes_per_chunk(gpu):
 
 def test_full_shape_48_layer_sequence(gpu):
     """All 48 layers x 16 steps run on the GPU; the oracle follows layers 0
-    and 47 (every append checked) and attention is compared at three steps."""
+    and 47 (every append checked); attention is compared on sampled rows at
+    steps 0 and 8 and over the whole output at the last step (ring wrapped)."""
     cfg = configs.get(4)
     R = Runner(4, cfg, oracle_layers=[0, 47])
     for step in range(cfg["steps"]):
@@ -150,9 +151,9 @@ def test_full_shape_48_layer_sequence(gpu):
         for layer in range(cfg["n_layers"]):
             out = torch.empty((R.T, R.H, R.D), dtype=torch.bfloat16, device="cuda")
             assert R.cache.attend(layer, out) == 0
-        if step in (0, 8, 15):
+        if step in (0, 8, cfg["steps"] - 1):
             for layer in (0, 47):
-                rows = sample_rows(R.T, 24, step * 7 + layer)
+                rows = None if step == cfg["steps"] - 1 else sample_rows(R.T, 24, step * 7 + layer)
                 g, o = R.attend(layer, rows=rows)
                 mx, rl = attn_errors(g, o)
                 assert mx <= ATOL_MAX and rl <= REL_L2, (step, layer, mx, rl)
