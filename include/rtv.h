@@ -15,7 +15,9 @@
  * granularity, the window or the mask.  This library implements: 3D axial
  * rotate-half RoPE over (frame t, grid row h, grid column w) segments of
  * head_dim, base rope_base, angles in fp64; OCP E4M3 codes with one fp32
- * scale amax/448 per (token, head) for Q, K and V; a ring of
+ * scale amax/448 per (token, head) for Q, K and V (an item whose amax is
+ * below 2^-119, where the fp32 reciprocal 448/amax would overflow, is stored
+ * as zero -- zero codes, scale 0 -- like an all-zero item); a ring of
  * window_frames + max_frames_per_chunk slots plus an optional pinned slot;
  * softmax(q.k / sqrt(head_dim)) attention of the chunk's queries over the
  * pinned frame, the window and the chunk's own frames, with no mask inside

@@ -96,13 +96,15 @@ __device__ __forceinline__ void unpack2(uint64_t r, float& a, float& b)
     asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(r));
 }
 
-// amax / 448, correctly rounded: the product with RN(1/448) corrected once by
-// its FMA residual (Markstein's correction step).  Checked against IEEE
-// division for every positive finite float from 2^-120 up; below that (a
-// subnormal quotient) the division itself is used.
+// Items with amax below this are stored as zero (zero codes, scale 0): the
+// fp32 reciprocal 448/amax would overflow there and turn zeros into NaN.
+constexpr float kMinAmax = 0x1p-119f;
+
+// amax / 448 for amax >= kMinAmax, correctly rounded: the product with
+// RN(1/448) corrected once by its FMA residual (Markstein's correction step),
+// which equals IEEE division for every positive finite float from 2^-120 up.
 __device__ __forceinline__ float div448(float a)
 {
-    if (!(a >= 0x1p-120f)) return __fdiv_rn(a, 448.f);
     constexpr float z = 1.0f / 448.0f;
     const float q0 = __fmul_rn(a, z);
     const float r = __fmaf_rn(-q0, 448.f, a);
@@ -185,10 +187,11 @@ __device__ __forceinline__ void append_rows_v(const AppendParams& p, unsigned in
                 for (int o = 8; o >= 1; o >>= 1)
                     amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
                 if (!row_ok || h >= H) continue;
-                const float inv = amax > 0.f ? __fdiv_rn(448.f, amax) : 0.f;
+                const bool keep = amax >= kMinAmax;
+                const float inv = keep ? __fdiv_rn(448.f, amax) : 0.f;
                 store_codes<E>(dst + (size_t)h * dst_step, y, inv);
                 if (lane16 == 0) {
-                    const float scale = div448(amax);
+                    const float scale = keep ? div448(amax) : 0.f;
                     sdst[(size_t)h * sdst_step] = scale;
                     atomicMax(&s_vmax[frame][h], __float_as_uint(scale));
                 }
@@ -302,7 +305,8 @@ __device__ __forceinline__ void append_rows_rope(const AppendParams& p, int tens
                 for (int o = 8; o >= 1; o >>= 1)
                     amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
                 if (!row_ok || h >= H) continue;
-                const float inv = amax > 0.f ? __fdiv_rn(448.f, amax) : 0.f;
+                const bool keep = amax >= kMinAmax;
+                const float inv = keep ? __fdiv_rn(448.f, amax) : 0.f;
                 uint8_t* d = dst + (size_t)h * dst_step;
                 if constexpr (P == 4) {
                     *reinterpret_cast<uint32_t*>(d + ea) =
@@ -313,7 +317,7 @@ __device__ __forceinline__ void append_rows_rope(const AppendParams& p, int tens
                     *reinterpret_cast<uint16_t*>(d + ea) = e4m3x2(mul2(ya[0], ya[1], inv));
                     *reinterpret_cast<uint16_t*>(d + eb) = e4m3x2(mul2(yb[0], yb[1], inv));
                 }
-                if (lane16 == 0) sdst[(size_t)h * sdst_step] = div448(amax);
+                if (lane16 == 0) sdst[(size_t)h * sdst_step] = keep ? div448(amax) : 0.f;
             }
         }
     }

@@ -91,8 +91,10 @@ __device__ __forceinline__ void quantise_store(float (&y)[kD], bool rope, const 
     float amax = 0.f;
 #pragma unroll
     for (int d = 0; d < kD; ++d) amax = fmaxf(amax, fabsf(y[d]));
-    const float inv = amax > 0.f ? __fdiv_rn(448.f, amax) : 0.f;
-    const float scale = __fdiv_rn(amax, 448.f);
+    // below 2^-119 the reciprocal would overflow: such an item is stored as zero
+    const bool keep = amax >= 0x1p-119f;
+    const float inv = keep ? __fdiv_rn(448.f, amax) : 0.f;
+    const float scale = keep ? __fdiv_rn(amax, 448.f) : 0.f;
 #pragma unroll
     for (int c = 0; c < kD / 16; ++c) {
         uint32_t w[4];

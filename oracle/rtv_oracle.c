@@ -175,10 +175,13 @@ void oracle_rope3d(const float* x, float* y, int D, int n_t, int n_h, int n_w,
 /*
  * Per (token, head) row of D values:
  *     amax  = max_d |x_d|                         (exact in fp32)
- *     inv   = fl(448 / amax)      (inv = 0 when amax = 0)
+ *     inv   = fl(448 / amax)      (inv = 0 when amax < 2^-119)
  *     code  = E4M3_RNE_sat(fl(x_d * inv))
- *     scale = fl(amax / 448)
- * so that decode(code) * scale approximates x_d.
+ *     scale = fl(amax / 448)      (scale = 0 when amax < 2^-119)
+ * so that decode(code) * scale approximates x_d.  Below 2^-119 the fp32
+ * reciprocal would overflow (448 / 2^-120 > FLT_MAX) and the product x_d * inv
+ * would turn zeros into NaN: such an item is stored as zero, as an all-zero
+ * item is (the reading: values under 2e-36 carry nothing the format can keep).
  */
 void oracle_quantize_row(const float* x, int D, uint8_t* codes, float* scale,
                          uint8_t* near_boundary)
@@ -190,14 +193,14 @@ void oracle_quantize_row(const float* x, int D, uint8_t* codes, float* scale,
         if (a > amax)
             amax = a;
     }
-    inv = amax > 0.0f ? 448.0f / amax : 0.0f;
+    inv = amax >= 0x1p-119f ? 448.0f / amax : 0.0f;
     for (d = 0; d < D; ++d) {
         float yv = x[d] * inv;
         codes[d] = oracle_e4m3_encode(yv);
         if (near_boundary)
             near_boundary[d] = oracle_e4m3_near_boundary(yv);
     }
-    *scale = amax / 448.0f;
+    *scale = amax >= 0x1p-119f ? amax / 448.0f : 0.0f;
 }
 
 /* -------------------------------------------------------------- append -- */

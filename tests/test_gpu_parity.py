@@ -15,7 +15,7 @@ import numpy as np
 import pytest
 import torch
 
-from kv_cache_serving_append_b200 import configs
+from kv_cache_serving_append_b200 import configs, synth
 from parity import ATOL_MAX, REL_L2, Runner, attn_errors, sample_rows
 
 pytestmark = pytest.mark.gpu
@@ -174,5 +174,68 @@ def test_bf16_output_small(gpu):
             assert np.all(np.abs(g - o) <= ATOL_MAX + 2.0 ** -8 * np.abs(o))
             _, rl = attn_errors(g, o)
             assert rl <= REL_L2
+        R.advance()
+    R.cache.close()
+
+
+def _degenerate(x: torch.Tensor, seed: int, large: bool) -> torch.Tensor:
+    """Seeded (row, head) items made degenerate: all zero (amax = 0), below
+    the reciprocal's range (amax < 2^-119: stored as zero), tiny but in range
+    (amax near 2^-108), a single nonzero element, and -- for Q and K -- large
+    (scores that outgrow the running reference: the softmax's redo and
+    rescale paths)."""
+    rows, H, _ = x.shape
+    g = torch.Generator().manual_seed(seed)
+    y = x.float().clone()
+    pick = torch.rand((rows, H), generator=g)
+    zero = pick < 0.02
+    tiny = (pick >= 0.02) & (pick < 0.04)
+    single = (pick >= 0.04) & (pick < 0.06)
+    small = (pick >= 0.07) & (pick < 0.09)
+    y[zero] = 0.0
+    y[tiny] = y[tiny] * 2.0 ** -126
+    y[small] = y[small] * 2.0 ** -110
+    keep = y[single][:, :1].clone()
+    y[single] = 0.0
+    y[single, :1] = keep
+    if large:
+        big = (pick >= 0.06) & (pick < 0.07)
+        y[big] = y[big] * 2.0 ** 8
+    return y.to(torch.bfloat16)
+
+
+@pytest.mark.gpu
+def test_degenerate_items(gpu):
+    """Zero, tiny, single-element and large (row, head) items: every append
+    code and scale bit-exact, attention over the whole output after the ring
+    wrapped."""
+    cfg = configs.get(2)
+
+    class DegenerateRunner(Runner):
+        def append(self, layer, step, n_frames, check=True):
+            q, k, v = synth.chunk(self.cfg_id, self.cfg, layer, step, n_frames)
+            base = 7919 * (step + 1) + 31 * layer
+            q = _degenerate(q, base, True)
+            k = _degenerate(k, base + 1, True)
+            v = _degenerate(v, base + 2, False)
+            st = self.cache.append(layer, q.to(self.device), k.to(self.device), v.to(self.device), n_frames)
+            assert st == 0, self.rtv.status_string(st)
+            if layer in self.ora.layers:
+                slots = self.ora.append(layer, synth.bf16_bits(q), synth.bf16_bits(k), synth.bf16_bits(v),
+                                        n_frames)
+                if check:
+                    self.check_append(layer, slots, n_frames)
+
+    R = DegenerateRunner(2, cfg)
+    last = cfg["window_frames"] + 2
+    for step in range(last + 1):
+        for layer in range(cfg["n_layers"]):
+            R.append(layer, step, 1)
+        if step in (0, last):
+            for layer in range(cfg["n_layers"]):
+                g, o = R.attend(layer)
+                mx, rl = attn_errors(g, o)
+                print(f"degenerate step {step} layer {layer}: max-abs {mx:.4g} rel-L2 {rl:.4g}")
+                assert mx <= ATOL_MAX and rl <= REL_L2, (step, layer, mx, rl)
         R.advance()
     R.cache.close()

@@ -184,3 +184,24 @@ def test_projection_definition_on_a_brute_force_case():
             import torch
             ref = torch.tensor([float(v)], dtype=torch.float32).to(torch.bfloat16).view(torch.int16).item() & 0xFFFF
             assert got[r, n] == ref, (r, n)
+
+
+def test_quantize_row_below_the_reciprocal_range_is_zero():
+    """Below amax = 2^-119 the fp32 reciprocal 448/amax would overflow (and a
+    zero times it would be NaN): such an item is stored as zero, scale 0.  At
+    and above 2^-119 the item quantises as usual, with its amax element on the
+    largest code and a finite, exact scale."""
+    rng = np.random.default_rng(12)
+    base = rng.standard_normal(128).astype(np.float32)
+    base[3] = 0.0
+    base /= np.abs(base).max()                       # amax = 1
+    rows = np.stack([base * np.float32(2.0 ** e) for e in (-126, -120, -119, -110)]).astype(np.float32)
+    codes, scales, _ = oracle.quantize_rows(rows)
+    for i in (0, 1):                                 # amax 2^-126, 2^-120: zero
+        assert np.all(codes[i] & 0x7F == 0) and scales[i] == 0.0
+    for i, e in ((2, -119), (3, -110)):              # amax 2^-119, 2^-110: quantised
+        amax = np.float32(2.0 ** e)
+        assert scales[i] == np.float32(amax / np.float32(448.0))
+        assert codes[i][np.argmax(np.abs(rows[i]))] & 0x7F == 0x7E
+        assert codes[i][3] & 0x7F == 0               # the zero element stays zero, not NaN
+        assert not np.any((codes[i] & 0x7F) == 0x7F)
