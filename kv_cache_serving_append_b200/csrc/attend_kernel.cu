@@ -47,8 +47,13 @@
 // V's per-token scale varies along PV's contraction dimension, so it is
 // folded into P.  Sv is a power of two at or above every V scale in the key
 // set (from the per-frame V-scale maxima the append kernel records); P =
-// p*scale_v/Sv stays <= 2^8 inside f16 range, and 1/Sv is folded into the
-// exponent so the row sum carries the same factor and O/l needs none.
+// p*scale_v/Sv stays below 2^15 (the redo bound), inside f16 range, and 1/Sv
+// is folded into the exponent so the row sum carries the same factor and O/l
+// needs none.
+//
+// When one CTA per (head, 256 query rows) would leave the last wave of the
+// GPU mostly idle, the host splits every unit's key range (grid z); each split
+// writes its unnormalised O and row statistics, and combine_kernel merges them.
 //
 // Registers: the block launches with 168 per thread; the four single-role
 // warps give theirs back (setmaxnreg 56) and the softmax warps take them
