@@ -63,8 +63,9 @@ def workload(cfg):
     M = F * T
     N = (cfg["pinned_frames"] + W + F) * T
     flops = 4.0 * M * N * D * H               # QK^T + PV, algorithmic
+    exps = float(M) * N * H                   # one exponential per score
     append_bytes = (3 * 2 * D + 3 * D + 12) * M * H   # bf16 in, codes + 3 fp32 scales out
-    return dict(T=T, H=H, D=D, M=M, N=N, flops=flops, append_bytes=append_bytes)
+    return dict(T=T, H=H, D=D, M=M, N=N, flops=flops, exps=exps, append_bytes=append_bytes)
 
 
 def ncu_traffic(kernel_file: str, summary: str):
@@ -694,6 +695,10 @@ def main():
 
     hbm_gbs, bf16_tf, bf16_tf_sus, peak_src = load_peaks()
     fp8_peak = 2.0 * bf16_tf
+    props = torch.cuda.get_device_properties(dev)
+    sm_count = props.multi_processor_count
+    sm_max_ghz = (clocks or {}).get("sm_max_mhz") or 1965.0
+    sm_max_ghz = sm_max_ghz / 1e3
     attn_tflops = wl["flops"] / (attend_ms * 1e-3) / 1e12
     append_gbs = wl["append_bytes"] / (append_ms * 1e-3) / 1e9
     us_per_step = us_per_layer_step(elapsed_ms, args.steps, world)
@@ -712,6 +717,14 @@ def main():
                                     "fp8:bf16 dense ratio)",
                      "traffic": ncu_traffic("attend_kernel.cu", "attend_full_shape_ncu.md"),
                      "algorithmic_flop_per_launch": wl["flops"]},
+        # context: the same attention call against its exponential throughput
+        # (one ex2 per score; 16 per clock per SM, measured by a probe; the
+        # SM count and the maximum SM clock of this device)
+        "roofline_exp": {"kernel": "rtv attend, softmax exponentials", "bound": "alu",
+                         "achieved": wl["exps"] / (attend_ms * 1e-3) / 1e9,
+                         "peak": 16 * sm_count * sm_max_ghz, "unit": "Gexp/s",
+                         "frac": wl["exps"] / (attend_ms * 1e-3) / 1e9 / (16 * sm_count * sm_max_ghz),
+                         "peak_source": "16 ex2/clock/SM x SMs x maximum SM clock"},
         "roofline_append": {"kernel": "rtv append (fused RoPE+amax+E4M3)", "bound": "hbm",
                             "achieved": append_gbs, "peak": hbm_gbs, "unit": "GB/s",
                             "frac": append_gbs / hbm_gbs,
